@@ -1,0 +1,551 @@
+// Tensor-core GEMM for the Newton-Schulz chain on sm_100a.
+//
+// Persistent, warp-specialised kernel: one CTA per SM, 256 threads.
+//   warp 0      TMA producer (one elected thread): A and B tiles into a
+//               4-stage shared-memory ring, 128-byte swizzle, no multicast
+//   warp 1      MMA issuer (one thread): tcgen05.mma kind::f16, 128x256x16
+//               per instruction, fp32 accumulator in TMEM
+//   warp 2      allocates / frees the 512 TMEM columns (two 128x256 fp32
+//               accumulators: the epilogue of tile i overlaps the mainloop of
+//               tile i+1)
+//   warps 4..7  epilogue: tcgen05.ld of 32x32 sub-tiles, fused
+//               alpha*acc + beta*C + gamma*I, narrowing store; for symmetric
+//               outputs the lower-triangle value is also written, transposed
+//               through shared memory, to the mirrored position.
+//
+// Symmetric outputs ("2. Symmetric GEMM Kernels" of the Dion3 page: a
+// triangular scheduler over lower tiles and a transposed-tile epilogue) are
+// scheduled over the 128x256 tiles that touch the lower triangle only.
+//
+// Every wait is bounded (mbar_wait_bounded): on expiry the kernel records
+// MUON_ERR_TIMEOUT, every role stops, in-flight copies and MMAs are drained
+// with bounded waits and TMEM is freed before the CTA exits.
+#include <cstring>
+#include <type_traits>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace muon {
+
+namespace tc {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int UMMA_K = 16;
+constexpr int A_STAGE = BM * BK * 2;  // 16 KB
+constexpr int B_STAGE = BN * BK * 2;  // 32 KB
+constexpr int THREADS = 256;
+constexpr int EPI_WARP0 = 4;
+constexpr int TMEM_COLS = 512;
+constexpr int EPI_BUF_WORDS = 32 * 33;  // per epilogue warp (padded 32x32 transpose)
+// Drains (in-flight copies and MMAs before exit) use their own bound, so that
+// a tiny configurable wait budget never lets a CTA exit with work in flight.
+constexpr uint64_t DRAIN_NS = 1000000000ull;
+constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_STAGE + B_STAGE) + 4 * EPI_BUF_WORDS * 4 +
+                           (2 * STAGES + 5) * 8 + 16;
+
+struct Group {
+  CUtensorMap tmA;
+  CUtensorMap tmB;
+  void* D;
+  const void* C;
+  const float* scale;
+  long long ldd, sD, ldc, sC;
+  int M, N, K, batch;
+  int a_mn, b_mn, sym, d_f32;
+  int alpha_pow, beta_pow;
+  float alpha, beta, gamma;
+  int tiles_m, tiles_n, tiles_per_batch, tile_begin;
+};
+
+struct Params {
+  Group g[kMaxGemmGroups];
+  int ngroups;
+  int total_tiles;
+  int* status;
+  unsigned long long timeout_ns;
+};
+
+struct Tile {
+  int g, b, m0, n0;
+};
+
+__host__ __device__ inline int sym_row_tiles(int i, int tiles_n) {
+  int c = (i * BM + BM - 1) / BN + 1;
+  return c < tiles_n ? c : tiles_n;
+}
+
+__device__ inline Tile decode(const Params& p, int tile) {
+  int gi = 0;
+  while (gi + 1 < p.ngroups && tile >= p.g[gi + 1].tile_begin) ++gi;
+  const Group& g = p.g[gi];
+  int local = tile - g.tile_begin;
+  int b = local / g.tiles_per_batch;
+  int t = local - b * g.tiles_per_batch;
+  int tm, tn;
+  if (!g.sym) {
+    tm = t % g.tiles_m;  // M fastest: concurrent CTAs share the B column block
+    tn = t / g.tiles_m;
+  } else {
+    int i = 0;
+    for (;;) {
+      int cnt = sym_row_tiles(i, g.tiles_n);
+      if (t < cnt) break;
+      t -= cnt;
+      ++i;
+    }
+    tm = i;
+    tn = t;
+  }
+  return Tile{gi, b, tm * BM, tn * BN};
+}
+
+__device__ __forceinline__ float powi(float s, int p) {
+  float r = 1.f;
+  for (int i = 0; i < p; ++i) r *= s;
+  return r;
+}
+
+template <typename T>
+__device__ __forceinline__ void store_row32(const Group& g, const Tile& t, int row, int c0, const float* v,
+                                            bool full_lower, bool any_lower) {
+  // Direct store of D[row, c0..c0+32). For symmetric outputs only elements
+  // with col <= row are written (full_lower: all 32 are).
+  if (row >= g.M || !any_lower) return;
+  if (g.d_f32) {
+    float* d = reinterpret_cast<float*>(g.D) + (long long)t.b * g.sD + (long long)row * g.ldd + c0;
+    if (full_lower) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4*>(d + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    } else {
+      for (int j = 0; j < 32; ++j)
+        if (c0 + j <= row) d[j] = v[j];
+    }
+  } else {
+    T* d = reinterpret_cast<T*>(g.D) + (long long)t.b * g.sD + (long long)row * g.ldd + c0;
+    if (full_lower) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) {
+        uint4 u;
+        u.x = Elem<T>::pack2(v[j], v[j + 1]);
+        u.y = Elem<T>::pack2(v[j + 2], v[j + 3]);
+        u.z = Elem<T>::pack2(v[j + 4], v[j + 5]);
+        u.w = Elem<T>::pack2(v[j + 6], v[j + 7]);
+        *reinterpret_cast<uint4*>(d + j) = u;
+      }
+    } else {
+      for (int j = 0; j < 32; ++j)
+        if (c0 + j <= row) d[j] = Elem<T>::from_f(v[j]);
+    }
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_STAGE;
+  uint32_t* sEpi = reinterpret_cast<uint32_t*>(sB + STAGES * B_STAGE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + 4 * EPI_BUF_WORDS);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4 * 32);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < p.ngroups; ++i) {
+      prefetch_tmap(&p.g[i].tmA);
+      prefetch_tmap(&p.g[i].tmB);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint64_t budget = p.timeout_ns;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------------
+    // TMA producer
+    // ------------------------------------------------------------------
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
+      const Tile t = decode(p, tile);
+      const Group& g = p.g[t.g];
+      const int nkb = (g.K + BK - 1) / BK;
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, budget, p.status)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[stage], A_STAGE + B_STAGE);
+        uint8_t* a = sA + stage * A_STAGE;
+        uint8_t* b = sB + stage * B_STAGE;
+        const int k0 = kb * BK;
+        if (!g.a_mn) {
+          tma_load_3d(a, &g.tmA, k0, t.m0, t.b, &full[stage]);
+        } else {
+          tma_load_3d(a, &g.tmA, t.m0, k0, t.b, &full[stage]);
+          tma_load_3d(a + 8192, &g.tmA, t.m0 + 64, k0, t.b, &full[stage]);
+        }
+        if (!g.b_mn) {
+          tma_load_3d(b, &g.tmB, k0, t.n0, t.b, &full[stage]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < BN / 64; ++j) tma_load_3d(b + j * 8192, &g.tmB, t.n0 + 64 * j, k0, t.b, &full[stage]);
+        }
+        ++issued;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+    }
+    // Drain: wait (bounded) until every copy issued into the ring landed.
+    int n = issued < STAGES ? issued : STAGES;
+    for (int i = 0; i < n; ++i) {
+      if (--stage < 0) {
+        stage = STAGES - 1;
+        phase ^= 1;
+      }
+      // the copies of the most recent use of `stage` completed phase `phase`
+      const uint32_t addr = smem_u32(&full[stage]);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(addr, phase)) {
+        if (globaltimer_ns() - t0 > DRAIN_NS) {
+          report(p.status, MUON_ERR_TIMEOUT);
+          break;
+        }
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------------
+    // MMA issuer
+    // ------------------------------------------------------------------
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
+    constexpr int fmt = sizeof(T) == 2 && std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.total_tiles && ok; tile += gridDim.x) {
+      const Tile t = decode(p, tile);
+      const Group& g = p.g[t.g];
+      const int nkb = (g.K + BK - 1) / BK;
+      const uint32_t idesc = idesc_f16(fmt, g.a_mn, g.b_mn, BM, BN);
+      // K-major: 8-row groups 1024 B apart, one K step = 32 B inside the
+      // swizzle atom. MN-major: 64-element MN atoms 8 KB apart (LBO), 8-row
+      // K groups 1024 B apart (SBO), one K step of 16 rows = 2048 B.
+      const uint32_t a_lbo = g.a_mn ? 8192u : 16u, b_lbo = g.b_mn ? 8192u : 16u;
+      const uint32_t a_kstep = g.a_mn ? 2048u : 32u, b_kstep = g.b_mn ? 2048u : 32u;
+      if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, budget, p.status)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait_bounded(&full[stage], phase, abort_flag, budget, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = a_base + stage * A_STAGE, b_addr = b_base + stage * B_STAGE;
+#pragma unroll
+        for (int k = 0; k < BK / UMMA_K; ++k) {
+          const uint64_t ad = smem_desc_sw128(a_addr + k * a_kstep, a_lbo, 1024);
+          const uint64_t bd = smem_desc_sw128(b_addr + k * b_kstep, b_lbo, 1024);
+          umma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+        }
+        umma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      umma_commit(&tfull[acc]);  // accumulator ready for the epilogue
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+    // Drain: every MMA issued by this thread completes before TMEM is freed.
+    umma_commit(drain);
+    const uint32_t addr = smem_u32(drain);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(addr, 0)) {
+      if (globaltimer_ns() - t0 > DRAIN_NS) {
+        report(p.status, MUON_ERR_TIMEOUT);
+        break;
+      }
+    }
+  } else if (warp >= EPI_WARP0) {
+    // ------------------------------------------------------------------
+    // Epilogue
+    // ------------------------------------------------------------------
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    uint32_t* buf = sEpi + q * EPI_BUF_WORDS;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
+      const Tile t = decode(p, tile);
+      const Group& g = p.g[t.g];
+      // every lane waits; the verdict is made warp-uniform so the warp-wide
+      // tcgen05.ld below never runs with part of the warp gone
+      const bool ok = mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, budget, p.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const float s = g.scale ? g.scale[t.b] : 1.f;
+      const float alpha = g.alpha * powi(s, g.alpha_pow);
+      const float beta = g.beta * powi(s, g.beta_pow);
+      const int r0 = t.m0 + q * 32;
+      const int row = r0 + lane;
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        const int c0 = t.n0 + ch * 32;
+        if (c0 >= g.N) break;                      // warp-uniform
+        if (g.sym && c0 > r0 + 31) break;          // whole sub-tile above the diagonal
+        uint32_t raw[32];
+        tmem_ld_32x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + ch * 32, raw);
+        tmem_wait_ld();
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = alpha * __uint_as_float(raw[j]);
+        if (g.beta != 0.f && row < g.M) {
+          const T* c = reinterpret_cast<const T*>(g.C) + (long long)t.b * g.sC + (long long)row * g.ldc + c0;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            const uint4 u = *reinterpret_cast<const uint4*>(c + j);
+            float2 f;
+            f = Elem<T>::unpack2(u.x); v[j] += beta * f.x; v[j + 1] += beta * f.y;
+            f = Elem<T>::unpack2(u.y); v[j + 2] += beta * f.x; v[j + 3] += beta * f.y;
+            f = Elem<T>::unpack2(u.z); v[j + 4] += beta * f.x; v[j + 5] += beta * f.y;
+            f = Elem<T>::unpack2(u.w); v[j + 6] += beta * f.x; v[j + 7] += beta * f.y;
+          }
+        }
+        if (g.gamma != 0.f) {
+          const int j = row - c0;
+          if (j >= 0 && j < 32) {
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj)
+              if (jj == j) v[jj] += g.gamma;
+          }
+        }
+        // round once to the stored type so the mirror holds identical values
+        if (!g.d_f32) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = Elem<T>::to_f(Elem<T>::from_f(v[j]));
+        }
+        const bool full_lower = !g.sym || (c0 + 31 <= row);
+        const bool any_lower = !g.sym || (c0 <= row);
+        store_row32<T>(g, t, row, c0, v, full_lower, any_lower);
+        if (g.sym && r0 + 31 > c0) {
+          // mirror: D[c, r] = D[r, c] for r > c, via a 32x32 transpose
+#pragma unroll
+          for (int j = 0; j < 32; ++j) buf[lane * 33 + j] = __float_as_uint(v[j]);
+          __syncwarp();
+          const int c = c0 + lane;  // mirrored row
+          if (c < g.N) {
+            float w[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) w[i] = __uint_as_float(buf[i * 33 + lane]);
+            const bool all = (r0 > c) && (r0 + 31 < g.M);
+            if (g.d_f32) {
+              float* d = reinterpret_cast<float*>(g.D) + (long long)t.b * g.sD + (long long)c * g.ldd + r0;
+              if (all) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(d + i) = make_float4(w[i], w[i + 1], w[i + 2], w[i + 3]);
+              } else {
+                for (int i = 0; i < 32; ++i)
+                  if (r0 + i > c && r0 + i < g.M) d[i] = w[i];
+              }
+            } else {
+              T* d = reinterpret_cast<T*>(g.D) + (long long)t.b * g.sD + (long long)c * g.ldd + r0;
+              if (all) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 8) {
+                  uint4 u;
+                  u.x = Elem<T>::pack2(w[i], w[i + 1]);
+                  u.y = Elem<T>::pack2(w[i + 2], w[i + 3]);
+                  u.z = Elem<T>::pack2(w[i + 4], w[i + 5]);
+                  u.w = Elem<T>::pack2(w[i + 6], w[i + 7]);
+                  *reinterpret_cast<uint4*>(d + i) = u;
+                }
+              } else {
+                for (int i = 0; i < 32; ++i)
+                  if (r0 + i > c && r0 + i < g.M) d[i] = Elem<T>::from_f(w[i]);
+              }
+            }
+          }
+          __syncwarp();
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+}  // namespace tc
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D map over [batch][outer][inner] with row stride ld and batch stride
+// (elements), box {64, box_outer, 1}, 128-byte swizzle, zero fill out of range.
+bool make_map(CUtensorMap* m, Op t, const void* base, int64_t inner, int64_t outer, int64_t batch, int64_t ld,
+              int64_t bstride, int box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const CUtensorMapDataType dt = t == Op::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)outer, (cuuint64_t)batch};
+  cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)(batch > 1 ? bstride : ld * outer) * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_outer, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  }
+  return n;
+}
+
+muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t timeout_ns, cudaStream_t s) {
+  if (ngroups < 1 || ngroups > kMaxGemmGroups || (t != Op::BF16 && t != Op::F16)) return MUON_ERR_INVALID_ARG;
+  tc::Params p;
+  memset(&p, 0, sizeof(p));
+  int total = 0;
+  int ng = 0;
+  for (int i = 0; i < ngroups; ++i) {
+    const GemmDesc& d = gd[i];
+    if (d.batch <= 0 || d.M <= 0 || d.N <= 0 || d.K <= 0) continue;
+    if (d.ldd % 64 || (d.beta != 0.f && d.ldc % 64)) return MUON_ERR_INVALID_ARG;
+    if (d.sym && d.M != d.N) return MUON_ERR_INVALID_ARG;
+    tc::Group& g = p.g[ng];
+    // A operand source: K-major [M][K], MN-major [K][M]
+    bool ok = d.a_mn ? make_map(&g.tmA, t, d.A, d.M, d.K, d.batch, d.lda, d.strideA, 64)
+                     : make_map(&g.tmA, t, d.A, d.K, d.M, d.batch, d.lda, d.strideA, tc::BM);
+    ok = ok && (d.b_mn ? make_map(&g.tmB, t, d.B, d.N, d.K, d.batch, d.ldb, d.strideB, 64)
+                       : make_map(&g.tmB, t, d.B, d.K, d.N, d.batch, d.ldb, d.strideB, tc::BN));
+    if (!ok) return MUON_ERR_CUDA;
+    g.D = d.D;
+    g.C = d.C;
+    g.scale = d.scale;
+    g.ldd = d.ldd;
+    g.sD = d.strideD;
+    g.ldc = d.ldc;
+    g.sC = d.strideC;
+    g.M = d.M;
+    g.N = d.N;
+    g.K = d.K;
+    g.batch = d.batch;
+    g.a_mn = d.a_mn;
+    g.b_mn = d.b_mn;
+    g.sym = d.sym;
+    g.d_f32 = d.d_f32;
+    g.alpha_pow = d.alpha_pow;
+    g.beta_pow = d.beta_pow;
+    g.alpha = d.alpha;
+    g.beta = d.beta;
+    g.gamma = d.gamma;
+    g.tiles_m = (d.M + tc::BM - 1) / tc::BM;
+    g.tiles_n = (d.N + tc::BN - 1) / tc::BN;
+    if (d.sym) {
+      int c = 0;
+      for (int i2 = 0; i2 < g.tiles_m; ++i2) c += tc::sym_row_tiles(i2, g.tiles_n);
+      g.tiles_per_batch = c;
+    } else {
+      g.tiles_per_batch = g.tiles_m * g.tiles_n;
+    }
+    g.tile_begin = total;
+    total += g.tiles_per_batch * d.batch;
+    ++ng;
+  }
+  if (ng == 0) return MUON_OK;
+  p.ngroups = ng;
+  p.total_tiles = total;
+  p.status = status;
+  p.timeout_ns = timeout_ns;
+
+  static bool attr_set[2] = {false, false};
+  const int ti = t == Op::BF16 ? 0 : 1;
+  const void* fn = t == Op::BF16 ? (const void*)tc::gemm_kernel<__nv_bfloat16> : (const void*)tc::gemm_kernel<__half>;
+  if (!attr_set[ti]) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES) != cudaSuccess)
+      return MUON_ERR_CUDA;
+    attr_set[ti] = true;
+  }
+  const int grid = total < num_sms() ? total : num_sms();
+  if (t == Op::BF16)
+    tc::gemm_kernel<__nv_bfloat16><<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(p);
+  else
+    tc::gemm_kernel<__half><<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
+}
+
+}  // namespace muon

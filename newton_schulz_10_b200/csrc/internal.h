@@ -1,0 +1,84 @@
+// Host-side interfaces between the libmuon translation units (not exported).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/muon.h"
+
+namespace muon {
+
+constexpr int kMaxGemmGroups = 4;
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // bound of every device wait
+
+// Operand element types of the GEMM chain.
+enum class Op { BF16 = 1, F16 = 2, F32 = 3 };
+
+inline size_t op_size(Op t) { return t == Op::F32 ? 4 : 2; }
+
+// Padded leading dimension (elements) of every internal matrix: a multiple of
+// 64 so that rows start on 128-byte boundaries (TMA strides, 16-byte vectors).
+inline int64_t pad_ld(int64_t cols) { return (cols + 63) / 64 * 64; }
+
+// One group of same-shape GEMMs, D_b = epilogue(Aop_b * Bop_b^T), b < batch.
+//   Aop[i,k] (M x K): a_mn = 0 -> A[i*lda + k]  (K-major, rows of A)
+//                     a_mn = 1 -> A[k*lda + i]  (MN-major)
+//   Bop[j,k] (N x K): b_mn = 0 -> B[j*ldb + k];  b_mn = 1 -> B[k*ldb + j]
+//   D = alpha*s^alpha_pow*acc + beta*s^beta_pow*C + gamma*I, s = scale[b]
+//   (s = 1 when scale is NULL); sym = 1: M == N and D is symmetric: only the
+//   lower triangle is computed and mirrored (D is then exactly symmetric).
+struct GemmDesc {
+  const void* A;
+  int64_t lda, strideA;
+  const void* B;
+  int64_t ldb, strideB;
+  void* D;
+  int64_t ldd, strideD;
+  const void* C;
+  int64_t ldc, strideC;
+  int M, N, K, batch;
+  int a_mn, b_mn, sym;
+  float alpha, beta, gamma;
+  const float* scale;
+  int alpha_pow, beta_pow;
+  int d_f32;  // tensor-core path only: write D as fp32 instead of the operand type
+};
+
+// Tensor-core GEMM (tcgen05 + TMEM + TMA), all groups in one persistent launch.
+// Operand type bf16 or f16. Returns MUON_OK or MUON_ERR_CUDA.
+muon_status tc_gemm(Op t, const GemmDesc* g, int ngroups, int* status, uint64_t timeout_ns, cudaStream_t s);
+
+// fp32 FFMA GEMM (no TF32), one group per launch.
+muon_status simt_gemm(const GemmDesc& g, cudaStream_t s);
+
+int num_sms();
+
+// One shape group of the Newton-Schulz chain: `count` matrices of
+// rows x cols in stored (row-major) orientation. A tall group (rows > cols)
+// is iterated in its transposed form through operand layouts; no copy.
+//   X[0], X[1]   [count][rows][ldx] operand ping-pong, ldx = pad_ld(cols);
+//                X[cur] holds the input on entry and the output on return
+//   xscale       per matrix: true X_0 = xscale[b] * stored X[cur] (NULL = 1)
+//   nb[]         [count][n][ldn] work matrices, n = min(rows, cols),
+//                ldn = pad_ld(n): 2 for the standard chain, 4 for Gram
+//   rho          Gram only: R is stored as rho * X X^T (keeps fp16 in range)
+struct NsGroup {
+  int64_t rows, cols;
+  int count;
+  void* X[2];
+  int cur;
+  const float* xscale;
+  void* nb[4];
+  float rho;
+};
+
+inline int ns_work_buffers(const muon_ns_params* p) { return p->gram ? 4 : 2; }
+
+// Run the chain (standard or Gram per p->gram) on up to kMaxGemmGroups
+// groups of operand type t; all groups share each launch.
+muon_status ns_run(Op t, NsGroup* gs, int ng, const muon_ns_params* p, int* status, uint64_t timeout_ns,
+                   cudaStream_t s);
+
+}  // namespace muon

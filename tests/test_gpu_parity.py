@@ -1,0 +1,266 @@
+"""Parity of the CUDA library (through its C ABI) with the fp64 oracle.
+
+Tolerances (relative Frobenius error): 1e-4 on fp32 paths, 2e-2 on
+bf16/fp16 Newton-Schulz outputs and on the weight change of a bf16 step;
+row-selection indices and the fp32 momentum state are compared bit for bit.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from newton_schulz_10_b200 import inputs
+from newton_schulz_10_b200 import muon as mu
+
+from gpu_util import COEFFS5, bf16_values, dev, gauss, host, rel
+
+pytestmark = pytest.mark.gpu
+
+TOL32 = 1e-4
+TOL16 = 2e-2
+
+
+@pytest.fixture(autouse=True)
+def _gpu(cuda):
+    yield
+    torch.cuda.synchronize()
+
+
+def status_of(ws) -> int:
+    torch.cuda.synchronize()
+    return int(ws[:4].view(torch.int32).item())
+
+
+# ---------------------------------------------------------------------------
+# ns_polar / gram_ns_polar
+# ---------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("shape", [(256, 1024), (300, 100), (17, 33), (1, 40), (64, 64)])
+def test_ns_polar_fp32(shape):
+    X = gauss(shape, 100 + shape[0])
+    Og, ws = mu.ns_polar(dev(X), mu.ns_params(compute=mu.F32))
+    assert status_of(ws) == mu.OK
+    assert rel(host(Og), O.newton_schulz(X.astype(np.float64), COEFFS5)) < TOL32
+
+
+BF16_SHAPES = [(128, 512), (200, 520), (520, 200), (64, 64), (300, 300), (1, 96), (96, 1), (8, 4096),
+               (768, 3072), (3072, 768), (130, 130), (256, 257)]
+
+
+@pytest.mark.parametrize("shape", BF16_SHAPES)
+def test_ns_polar_bf16(shape):
+    X = gauss(shape, 200 + shape[0] + shape[1])
+    Og, ws = mu.ns_polar(dev(X), mu.ns_params(compute=mu.BF16), out_dtype=torch.float32)
+    assert status_of(ws) == mu.OK
+    assert rel(host(Og), O.newton_schulz(X.astype(np.float64), COEFFS5)) < TOL16
+
+
+def test_ns_polar_bf16_input_output():
+    X32 = gauss((192, 640), 7)
+    Xb = dev(X32, torch.bfloat16)
+    Og, ws = mu.ns_polar(Xb, mu.ns_params(compute=mu.BF16))
+    assert Og.dtype == torch.bfloat16 and status_of(ws) == mu.OK
+    assert rel(host(Og), O.newton_schulz(bf16_values(X32), COEFFS5)) < TOL16
+
+
+@pytest.mark.parametrize("compute", [mu.F16, mu.BF16, mu.F32])
+@pytest.mark.parametrize("restart", [3, 0])
+@pytest.mark.parametrize("shape", [(256, 1024), (200, 520), (520, 200), (96, 96)])
+def test_gram_ns_polar(compute, restart, shape):
+    X = gauss(shape, 300 + shape[0])
+    p = mu.ns_params(gram=True, restart_at=restart, compute=compute)
+    Og, ws = mu.gram_ns_polar(dev(X), p, out_dtype=torch.float32)
+    assert status_of(ws) == mu.OK
+    want = O.gram_newton_schulz(X.astype(np.float64), COEFFS5, restart_at=restart)
+    assert rel(want, O.newton_schulz(X.astype(np.float64), COEFFS5)) < 1e-9
+    assert rel(host(Og), want) < (TOL32 if compute == mu.F32 else TOL16)
+
+
+@pytest.mark.parametrize("gram", [False, True])
+def test_spectrum_matrix(gram):
+    """Singular values log-uniform in [1e-4, 1] (the spectrum workload, small)."""
+    X, _ = inputs.spectrum_matrix(256, 1024, -4.0, seed=31)
+    X32 = X.astype(np.float32)
+    p = mu.ns_params(gram=gram, compute=mu.F16 if gram else mu.BF16)
+    Og, ws = mu.ns_polar(dev(X32, torch.bfloat16), p, out_dtype=torch.float32)
+    assert status_of(ws) == mu.OK
+    Xb = bf16_values(X32)
+    want = O.newton_schulz(Xb, COEFFS5)
+    assert rel(host(Og), want) < TOL16
+
+
+def test_time_varying_coefficients():
+    coeffs = [(4.0, -5.0, 2.1), (3.4445, -4.7750, 2.0315), (3.0, -3.5, 1.6), (2.0, -1.5, 0.55)]
+    X = gauss((128, 384), 41)
+    for gram in (False, True):
+        p = mu.ns_params(T=4, coeffs=coeffs, gram=gram, compute=mu.F32)
+        Og, ws = mu.ns_polar(dev(X), p)
+        assert rel(host(Og), O.newton_schulz(X.astype(np.float64), coeffs)) < TOL32
+
+
+def test_zero_matrix_gives_zero():
+    Og, ws = mu.ns_polar(torch.zeros(64, 128, device="cuda"), mu.ns_params())
+    assert status_of(ws) == mu.OK and torch.count_nonzero(Og).item() == 0
+
+
+# ---------------------------------------------------------------------------
+# select_rows / normuon_scale
+# ---------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("norm", [mu.NORM_L1, mu.NORM_L2])
+def test_select_rows_exact(norm):
+    g = inputs.rng(55, 0)
+    for n, m in [(1000, 300), (64, 33), (8192, 256), (5, 4)]:
+        M = g.standard_normal((n, m)).astype(np.float32)
+        M[n // 2] = M[0]          # exact ties
+        M[n - 1] = -M[1]
+        Md = dev(M)
+        for k in sorted({1, max(1, n // 4), n // 2 or 1, n}):
+            idx = mu.select_rows(Md, k, norm).cpu().numpy()
+            want = O.select_rows(M, k, "l1" if norm == mu.NORM_L1 else "l2")
+            assert np.array_equal(idx, want), (n, m, k)
+
+
+def test_normuon_scale_fp32():
+    g = inputs.rng(56, 0)
+    Om = g.standard_normal((300, 130)).astype(np.float32)
+    v0 = (g.random(300) * 0.01).astype(np.float32)
+    v = dev(v0)
+    scale = mu.normuon_scale(dev(Om), v, beta2=0.9, eps=1e-8)
+    v_want, s_want = O.normuon(Om.astype(np.float64), v0.astype(np.float64), 0.9, 1e-8)
+    assert rel(host(v), v_want) < 1e-5
+    assert rel(host(scale), s_want) < 1e-5
+    # with a row map: only mapped entries of v change
+    v2 = dev(np.zeros(500, np.float32))
+    rows = dev(np.arange(0, 600, 2)[:300].astype(np.int32), torch.int32)
+    mu.normuon_scale(dev(Om), v2, beta2=0.9, eps=1e-8, rows=rows)
+    hv = host(v2)
+    assert np.all(hv[1::2] == 0)
+    v_want2, _ = O.normuon(Om.astype(np.float64), np.zeros(300), 0.9, 1e-8)
+    assert rel(hv[0::2][:250], v_want2[:250]) < 1e-5
+
+
+# ---------------------------------------------------------------------------
+# muon_step
+# ---------------------------------------------------------------------------
+
+
+def make_state(shapes, seed, m_std=0.0):
+    out = []
+    for i, (r, c) in enumerate(shapes):
+        W = inputs.gaussian((r, c), 0.02, seed + i, 0)
+        G = inputs.gaussian((r, c), 1e-3, seed + i, 1)
+        M = inputs.gaussian((r, c), m_std, seed + i, 2) if m_std else np.zeros((r, c), np.float32)
+        v = np.zeros(r, np.float32)
+        out.append((W, M, G, v))
+    return out
+
+
+def run_step(state, p):
+    dmats = [(dev(W), dev(M), dev(G), dev(v)) for (W, M, G, v) in state]
+    s = mu.muon_step(dmats, p)
+    st = s.device_status()
+    return [(host(a), host(b), host(d)) for (a, b, _, d) in dmats], st
+
+
+def check_step(state, got, sp: O.StepParams, tol, label=""):
+    for (W, M, G, v), (Wg, Mg, vg) in zip(state, got):
+        want = O.muon_step(W, M, G, v, sp)
+        assert np.array_equal(Mg.astype(np.float32), want["M"]), f"{label} momentum state differs"
+        dW = Wg - W.astype(np.float64)
+        dW_want = want["W"].astype(np.float64) - W.astype(np.float64)
+        assert rel(dW, dW_want) < tol, (label, W.shape, rel(dW, dW_want))
+        if sp.normuon:
+            assert rel(vg, want["v"]) < tol
+        if sp.k is not None:
+            changed = np.where(np.any(Wg != W, axis=1))[0]
+            assert set(changed) <= set(want["idx"].tolist())
+
+
+def test_step_fp32_single():
+    state = make_state([(256, 1024)], 1000, m_std=1e-3)
+    p = mu.step_params(ns=mu.ns_params(compute=mu.F32))
+    got, st = run_step(state, p)
+    assert st == mu.OK
+    check_step(state, got, O.StepParams(), TOL32)
+
+
+MIXED = [(128, 128), (128, 128), (128, 384), (384, 128), (100, 260), (260, 100), (64, 64)]
+
+
+@pytest.mark.parametrize("gram,compute", [(False, mu.BF16), (True, mu.F16), (True, mu.BF16), (False, mu.F32)])
+def test_step_batched(gram, compute):
+    state = make_state(MIXED, 2000, m_std=2e-3)
+    p = mu.step_params(ns=mu.ns_params(gram=gram, compute=compute))
+    got, st = run_step(state, p)
+    assert st == mu.OK
+    check_step(state, got, O.StepParams(gram=gram), TOL32 if compute == mu.F32 else TOL16)
+
+
+@pytest.mark.parametrize("compute", [mu.BF16, mu.F32])
+def test_step_normuon(compute):
+    state = make_state(MIXED[:5], 3000, m_std=2e-3)
+    for i, s in enumerate(state):
+        s[3][:] = (inputs.rng(7 + i, 0).random(s[3].shape[0]) * 1e-4).astype(np.float32)
+    p = mu.step_params(ns=mu.ns_params(compute=compute), normuon=True, beta2=0.95, normuon_eps=1e-8)
+    got, st = run_step(state, p)
+    assert st == mu.OK
+    check_step(state, got, O.StepParams(normuon=True), TOL32 if compute == mu.F32 else TOL16)
+
+
+@pytest.mark.parametrize("norm", ["l1", "l2"])
+@pytest.mark.parametrize("frac", [(1, 4), (1, 2), (1, 1)])
+def test_step_dion3(norm, frac):
+    shapes = [(256, 512), (512, 256), (200, 96)]
+    state = make_state(shapes, 4000, m_std=3e-3)
+    p = mu.step_params(ns=mu.ns_params(gram=True, compute=mu.F16), dion3=True, frac=frac, normuon=True,
+                       select_norm=mu.NORM_L1 if norm == "l1" else mu.NORM_L2)
+    got, st = run_step(state, p)
+    assert st == mu.OK
+    for (W, M, G, v), g in zip(state, got):
+        k = O.rows_for_fraction(W.shape[0], *frac)
+        check_step([(W, M, G, v)], [g], O.StepParams(gram=True, normuon=True, k=k, select_norm=norm), TOL16,
+                   f"dion3 {norm} {frac}")
+
+
+def test_step_zero_and_empty():
+    state = make_state([(64, 128)], 5000)
+    state[0][2][:] = 0  # zero gradient, zero momentum
+    got, st = run_step(state, mu.step_params())
+    assert st == mu.OK
+    assert np.array_equal(got[0][0], state[0][0].astype(np.float64))
+
+
+def test_step_nonfinite_reported():
+    state = make_state([(64, 128)], 5100)
+    state[0][2][3, 5] = np.nan
+    _, st = run_step(state, mu.step_params())
+    assert st == mu.ERR_NONFINITE
+
+
+def test_step_deterministic_and_resumable():
+    """Two steps in one go equal one step, a save/reload of the state, and a
+    second step (bit for bit): fixed reduction orders, no float atomics."""
+    shapes = [(128, 384), (384, 128)]
+    state = make_state(shapes, 6000, m_std=1e-3)
+    G2 = [inputs.gaussian(s, 1e-3, 6100 + i, 1) for i, s in enumerate(shapes)]
+    p = mu.step_params(normuon=True)
+    d1 = [(dev(W), dev(M), dev(G), dev(v)) for (W, M, G, v) in state]
+    s1 = mu.muon_step(d1, p)
+    for i, g in enumerate(G2):
+        d1[i][2].copy_(dev(g))
+    s1()
+    ref = [tuple(host(t) for t in (a, b, d)) for (a, b, _, d) in d1]
+    # run 1 step, checkpoint to host, restore into fresh buffers, run step 2
+    d2 = [(dev(W), dev(M), dev(G), dev(v)) for (W, M, G, v) in state]
+    mu.muon_step(d2, p)
+    saved = [tuple(t.cpu().clone() for t in m) for m in d2]
+    d3 = [tuple(t.cuda() for t in m) for m in saved]
+    for i, g in enumerate(G2):
+        d3[i][2].copy_(dev(g))
+    mu.muon_step(d3, p)
+    for r, (a, b, _, d) in zip(ref, d3):
+        assert np.array_equal(r[0], host(a)) and np.array_equal(r[1], host(b)) and np.array_equal(r[2], host(d))
