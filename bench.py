@@ -1,0 +1,530 @@
+"""Benchmark of the Muon optimizer step on B200 (one JSON line on rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gpt124m|...] [--impl ours|reference]
+
+Default workload: the GPT-124M-shaped layer set (12 layers x {4 x 768x768,
+768x3072, 3072x768}), fp32 W/M/G, Newton-Schulz in bf16 with T = 5, one
+batched step per iteration. Under torchrun every rank runs its own replica of
+the step (the path has no cross-matrix exchange); the reported time is the
+max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only other arm) on a bounded
+sample of the same workload, scaled to the whole step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from newton_schulz_10_b200 import inputs  # noqa: E402
+
+METRIC = "Muon optimizer step ms/step; NS GEMM TFLOP/s vs B200 bf16 peak; HBM GB/s"
+COEFFS = (3.4445, -4.7750, 2.0315)
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+
+WORKLOADS = {
+    "single256x1024": dict(desc="single 256x1024 fp32 matrix, fp32 Newton-Schulz (T=5), one step",
+                           compute="f32", gram=False, normuon=False, dion3=None),
+    "gpt124m": dict(desc="GPT-124M layer set: 12 x (4 x 768x768, 768x3072, 3072x768), bf16 NS T=5",
+                    compute="bf16", gram=False, normuon=False, dion3=None),
+    "dion3_8192x28672": dict(desc="8192x28672, Dion3 f=1/4 (l1 rows) + NorMuon, Gram NS fp16 (restart 3), T=5",
+                             compute="f16", gram=True, normuon=True, dion3=(1, 4)),
+    "llama7b": dict(desc="Llama-7B layer set: 32 x (4 x 4096x4096, 4096x14336, 14336x4096), bf16 NS T=5",
+                    compute="bf16", gram=False, normuon=False, dion3=None),
+    "llama7b_normuon": dict(desc="Llama-7B layer set, bf16 NS T=5, NorMuon on",
+                            compute="bf16", gram=False, normuon=True, dion3=None),
+    "spectrum4096x16384": dict(desc="one 4096x16384 bf16 matrix, singular values log-uniform in [1e-4, 1]: "
+                                    "Gram NS (fp16, restart 3) vs standard NS (bf16 and fp16), T=5",
+                               compute="f16", gram=True, normuon=False, dion3=None),
+}
+
+
+def ns_flops(n, m, T, gram, restart_at=3):
+    """The page's FLOP counts with symmetric GEMMs: standard T(3 alpha + 1) n^3,
+    Gram (4T + 3 alpha - 3) n^3, plus 3(alpha - 1) n^3 per restart."""
+    if not gram:
+        return T * (3 * m * n * n + n ** 3)
+    f = 4 * T * n ** 3 + 3 * m * n * n - 3 * n ** 3
+    if restart_at and 1 < restart_at <= T:
+        f += 3 * m * n * n - 3 * n ** 3
+    return f
+
+
+def specs_for(name: str):
+    if name == "spectrum4096x16384":
+        return [inputs.MatrixSpec(4096, 16384, 3000, "x")]
+    if name == "single256x1024":
+        return [inputs.MatrixSpec(256, 1024, 1000, "x")]
+    if name == "gpt124m":
+        return inputs.gpt124m_layer_set()
+    if name == "dion3_8192x28672":
+        return [inputs.MatrixSpec(8192, 28672, 4000, "x")]
+    if name.startswith("llama7b"):
+        return inputs.llama7b_layer_set()
+    raise ValueError(name)
+
+
+def host_state(spec: inputs.MatrixSpec, workload: str):
+    """Seeded W, M0 = 0, G for one matrix (fp32, host)."""
+    shape = (spec.rows, spec.cols)
+    if workload == "single256x1024":
+        W = inputs.gaussian(shape, 1.0, spec.seed, inputs.W_STREAM)
+        G = inputs.gaussian(shape, 1.0, spec.seed, inputs.G_STREAM)
+    elif workload == "gpt124m":
+        W = inputs.gaussian(shape, 0.02, spec.seed, inputs.W_STREAM)
+        G = inputs.gaussian(shape, 1e-3, spec.seed, inputs.G_STREAM)
+    else:
+        W = inputs.gaussian(shape, 0.02, spec.seed, inputs.W_STREAM)
+        G = inputs.student_t3(shape, 1e-3, spec.seed, inputs.G_STREAM)
+    return W, np.zeros(shape, np.float32), G
+
+
+def device_state(spec, workload, torch, gen_on_device: bool):
+    shape = (spec.rows, spec.cols)
+    if not gen_on_device:
+        W, M, G = host_state(spec, workload)
+        return [torch.from_numpy(a).cuda() for a in (W, M, G)]
+    # large sets: same distributions drawn on the device (torch Philox, seeded per matrix)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(spec.seed)
+    W = torch.randn(shape, device="cuda", generator=g) * 0.02
+    z = torch.randn(shape, device="cuda", generator=g)
+    chi = torch.zeros(shape, device="cuda")
+    for _ in range(3):
+        chi.add_(torch.randn(shape, device="cuda", generator=g).square_())
+    G = z.div_(chi.div_(3.0).sqrt_()).mul_(1e-3)
+    del chi
+    return [W, torch.zeros(shape, device="cuda"), G]
+
+
+def step_params(mu, cfg, rows_hint=None):
+    comp = {"f32": mu.F32, "bf16": mu.BF16, "f16": mu.F16}[cfg["compute"]]
+    ns = mu.ns_params(T=5, coeffs=COEFFS, gram=cfg["gram"], restart_at=3, compute=comp)
+    return mu.step_params(mu=0.95, lr=0.02, ns=ns, normuon=cfg["normuon"], beta2=0.95, normuon_eps=1e-8,
+                          dion3=cfg["dion3"] is not None, frac=cfg["dion3"] or (1, 1), select_norm=mu.NORM_L1)
+
+
+# ---------------------------------------------------------------------------
+# measurement helpers
+# ---------------------------------------------------------------------------
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((ts, float(parts[0]), float(parts[1]), parts[3:]))
+            except ValueError:
+                continue
+        inside = [r for r in rows if t0 <= r[0] <= t1] or rows
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3][1:5]) if v.lower() == "active"})
+        return {"sm_mhz": float(np.median([r[1] for r in inside])), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside),
+                "in_region": any(t0 <= r[0] <= t1 for r in rows)}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from newton_schulz_10_b200 import muon as mu
+
+    torch.cuda.set_device(local_rank)
+    cfg = WORKLOADS[args.workload]
+    specs = specs_for(args.workload)
+    big = sum(s.rows * s.cols for s in specs) > 1_000_000_000
+    state = []
+    for s in specs:
+        W, M, G = device_state(s, args.workload, torch, gen_on_device=big)
+        v = torch.zeros(s.rows, device="cuda")
+        state.append((W, M, G, v))
+    p = step_params(mu, cfg)
+    step = mu.Step([tuple(x) for x in state], p)
+    stream = torch.cuda.current_stream()
+    elems = sum(s.rows * s.cols for s in specs)
+
+    for _ in range(args.warmup):
+        step(stream)
+    torch.cuda.synchronize()
+    status = step.device_status()
+
+    # --- device-resident timing -------------------------------------------
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = mu.kernel_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        t0 = time.time()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step(stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t1 = time.time()
+    launches = mu.kernel_launch_count() - n0
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        tt = torch.tensor([ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    clocks = clk.summary(t0, t1)
+
+    # --- per-phase profile (separate, untimed run) --------------------------
+    prof = step.profiled(stream)
+
+    # --- end to end through host buffers ------------------------------------
+    # each step: H2D copy of that step's gradients from pinned memory, the
+    # step, D2H copy of the updated weights into pinned memory
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except ImportError:
+        avail = 1 << 62
+    if 2 * 4 * elems > 0.5 * avail:
+        raise SystemExit("not enough host memory for the end-to-end arm")
+    hostG = [torch.empty_like(G, device="cpu").pin_memory() for (_, _, G, _) in state]
+    hostW = [torch.empty_like(W, device="cpu").pin_memory() for (W, _, _, _) in state]
+    for hg, (_, _, G, _) in zip(hostG, state):
+        hg.copy_(G)
+    e2e_steps = max(1, min(args.steps, 20 if not big else 3))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        for hg, (_, _, G, _) in zip(hostG, state):
+            G.copy_(hg, non_blocking=True)
+        step(stream)
+        for hw, (W, _, _, _) in zip(hostW, state):
+            hw.copy_(W, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / e2e_steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+
+    peaks, peak_kind = measured_peaks()
+    long_step = ms > 100.0
+    tensor_peak = peaks["bf16_tflops_sustained" if long_step else "bf16_tflops"]
+    if cfg["compute"] == "f32":
+        roof = None
+    else:
+        achieved = prof.ns_flops / (prof.ms_ns * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 NS chain)", "achieved": round(achieved, 1),
+                "peak": tensor_peak, "unit": "TFLOP/s", "frac": round(achieved / tensor_peak, 4),
+                "traffic": None, "peak_source": f"{peak_kind} {'sustained' if long_step else 'burst'} bf16",
+                "flops_per_step_algorithmic": prof.ns_flops, "flops_per_step_executed": prof.ns_flops_executed,
+                "gemm_launches_per_step": prof.gemm_launches,
+                "achieved_executed": round(prof.ns_flops_executed / (prof.ms_ns * 1e-3) / 1e12, 1)}
+    hbm = peaks["hbm_gbs"]
+    phases = {k: round(getattr(prof, k), 4) for k in ("ms_total", "ms_prologue", "ms_ns", "ms_normuon", "ms_update")}
+    phases["prologue_gbs"] = round(prof.bytes_prologue / (prof.ms_prologue * 1e-3) / 1e9, 1) if prof.ms_prologue else None
+    upd_ms = prof.ms_update + prof.ms_normuon
+    phases["update_gbs"] = round(prof.bytes_update / (upd_ms * 1e-3) / 1e9, 1) if upd_ms else None
+    phases["hbm_peak_gbs"] = hbm
+    phases["kernel_launches_per_step"] = prof.kernel_launches
+
+    out = {
+        "metric": METRIC, "value": round(ms, 4), "unit": "ms/step", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg["compute"], "data": "synthetic",
+        "config": {"workload": args.workload, "description": cfg["desc"], "matrices": len(specs),
+                   "elements": elems, "state_bytes": 12 * elems,
+                   "l2": "inputs larger than L2 (fp32 W, M, G resident in HBM)",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": roof,
+        "phases": phases,
+        "e2e": {"value": round(e2e_ms, 3), "unit": "ms/step", "h2d_bytes_per_step": 4 * elems,
+                "d2h_bytes_per_step": 4 * elems, "what": "G pinned-host->device, step, W device->pinned-host"},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "device_status": mu.status_str(status),
+    }
+    return out
+
+
+def run_spectrum(args, rank, world, local_rank):
+    """Gram vs standard Newton-Schulz on the 4096 x 16384 spectrum matrix."""
+    import torch
+    import torch.distributed as dist
+
+    from newton_schulz_10_b200 import muon as mu
+
+    torch.cuda.set_device(local_rank)
+    X, _ = inputs.spectrum_matrix(4096, 16384, -4.0, seed=3000)
+    Xd = torch.from_numpy(X.astype(np.float32)).cuda().to(torch.bfloat16)
+    del X
+    n, m = 4096, 16384
+    variants = [("gram_f16", mu.ns_params(gram=True, restart_at=3, compute=mu.F16), True),
+                ("standard_bf16", mu.ns_params(compute=mu.BF16), False),
+                ("standard_f16", mu.ns_params(compute=mu.F16), False)]
+    stream = torch.cuda.current_stream()
+    res = {}
+    clocks = None
+    launches = 0
+    for name, p, gram in variants:
+        O, ws = mu.ns_polar(Xd, p, out_dtype=torch.bfloat16)
+        for _ in range(args.warmup):
+            mu.ns_polar(Xd, p, out_dtype=torch.bfloat16, ws=ws)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        n0 = mu.kernel_launch_count()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local_rank) as clk:
+            t0 = time.time()
+            e0.record(stream)
+            for _ in range(args.steps):
+                O, _ = mu.ns_polar(Xd, p, out_dtype=torch.bfloat16, ws=ws)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            t1 = time.time()
+        ms = e0.elapsed_time(e1) / args.steps
+        if world > 1:
+            tt = torch.tensor([ms], device="cuda")
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ms = float(tt.item())
+        if name == "gram_f16":
+            clocks = clk.summary(t0, t1)
+            launches = mu.kernel_launch_count() - n0
+        Of = O.float()
+        orth = float(torch.linalg.matrix_norm(Of @ Of.T - torch.eye(n, device="cuda")).item())
+        fl = ns_flops(n, m, 5, gram)
+        res[name] = {"ms": round(ms, 3), "tflops_algorithmic": round(fl / (ms * 1e-3) / 1e12, 1),
+                     "orthogonality_error_fro": round(orth, 4),
+                     "status": mu.status_str(int(ws[:4].view(torch.int32).item()))}
+        del O, ws
+    peaks, kind = measured_peaks()
+    g = res["gram_f16"]
+    peak = peaks["bf16_tflops"]  # fp16 and bf16 share the dense tensor-core rate
+    cfg = WORKLOADS[args.workload]
+    return {
+        "metric": METRIC, "value": g["ms"], "unit": "ms/step", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": g["ms"], "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": args.workload, "description": cfg["desc"], "step": "one gram_ns_polar call",
+                   "l2": "operands 128 MiB bf16 input + 256 MiB working set, larger than L2"},
+        "roofline": {"bound": "tensor", "kernel": "gemm_kernel (Gram NS chain)", "achieved": g["tflops_algorithmic"],
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(g["tflops_algorithmic"] / peak, 4),
+                     "traffic": None, "peak_source": f"{kind} burst bf16 (fp16 has the same dense rate)"},
+        "variants": res,
+        "speedup_gram_vs_standard_bf16": round(res["standard_bf16"]["ms"] / g["ms"], 3),
+        "e2e": None, "gpu_launches": launches, "clocks": clocks,
+    }
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+
+
+def oracle_sample(workload: str, budget_s: float):
+    """Time the oracle on a bounded sample of the workload; returns
+    (ms per full step, description of the sample, threads used)."""
+    import oracle
+
+    cfg = WORKLOADS[workload]
+    specs = specs_for(workload)
+    if workload == "spectrum4096x16384":
+        t = time.perf_counter()
+        X, _ = inputs.spectrum_matrix(1024, 4096, -4.0, seed=3000)
+        t_gen = time.perf_counter() - t
+        t = time.perf_counter()
+        oracle.gram_newton_schulz(X, (COEFFS,) * 5, 1e-7, 3)
+        dt = time.perf_counter() - t
+        scale = ns_flops(4096, 16384, 5, True) / ns_flops(1024, 4096, 5, True)
+        return 1e3 * dt * scale, (f"oracle gram_newton_schulz on a 1024x4096 matrix of the same spectrum, "
+                                  f"{dt:.1f} s, scaled x{scale:.0f} by the Gram FLOP formula"), threads_used()
+    sp = oracle.StepParams(mu=0.95, lr=0.02, coeffs=(COEFFS,) * 5, gram=cfg["gram"], normuon=cfg["normuon"])
+    total_flops = 0.0
+    for s in specs:
+        n, m = min(s.rows, s.cols), max(s.rows, s.cols)
+        if cfg["dion3"] is not None:
+            n = min(oracle.rows_for_fraction(s.rows, *cfg["dion3"]), s.cols)
+            m = max(oracle.rows_for_fraction(s.rows, *cfg["dion3"]), s.cols)
+        total_flops += oracle.flops_standard_dense(n, m, 5)
+    done_flops, t_sum, names = 0.0, 0.0, []
+    # one matrix of each distinct shape first, then more until the budget is used
+    seen, first, rest = set(), [], []
+    for i, s in enumerate(specs):
+        (rest if (s.rows, s.cols) in seen else first).append(i)
+        seen.add((s.rows, s.cols))
+    order = first + rest
+    for i in order:
+        s = specs[i]
+        W, M, G = host_state(s, workload)
+        v = np.zeros(s.rows, np.float32)
+        p = sp
+        if cfg["dion3"] is not None:
+            p = oracle.StepParams(**{**sp.__dict__, "k": oracle.rows_for_fraction(s.rows, *cfg["dion3"])})
+        t = time.perf_counter()
+        oracle.muon_step(W, M, G, v, p)
+        t_sum += time.perf_counter() - t
+        n, m = min(s.rows, s.cols), max(s.rows, s.cols)
+        if cfg["dion3"] is not None:
+            k = oracle.rows_for_fraction(s.rows, *cfg["dion3"])
+            n, m = min(k, s.cols), max(k, s.cols)
+        done_flops += oracle.flops_standard_dense(n, m, 5)
+        names.append(s.name)
+        if t_sum > budget_s:
+            break
+    scale = total_flops / done_flops
+    desc = (f"oracle muon_step on {len(names)} of {len(specs)} matrices ({', '.join(names[:6])}"
+            f"{', ...' if len(names) > 6 else ''}), {t_sum:.1f} s, scaled x{scale:.2f} by NS FLOPs to the whole step")
+    return 1e3 * t_sum * scale, desc, threads_used()
+
+
+def threads_used():
+    for var in ("OPENBLAS_NUM_THREADS", "OMP_NUM_THREADS"):
+        if os.environ.get(var):
+            return int(os.environ[var])
+    return os.cpu_count()
+
+
+def run_reference(args):
+    cfg = WORKLOADS[args.workload]
+    per_step_budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(args.workload, per_step_budget)
+    vals = []
+    desc = ""
+    for _ in range(args.steps):
+        v, desc, cores = oracle_sample(args.workload, per_step_budget)
+        vals.append(v)
+    ms = float(np.mean(vals))
+    return {"impl": "reference", "metric": METRIC, "value": round(ms, 2), "unit": "ms/step", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "description": cfg["desc"]},
+            "cpu_baseline": {"value": round(ms, 2), "unit": "ms/step", "cores": threads_used(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": round(ms, 2), "unit": "ms/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt124m")
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    if args.workload == "spectrum4096x16384":
+        out = run_spectrum(args, rank, world, local_rank)
+    else:
+        out = run_ours(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ms, desc, cores = oracle_sample(args.workload, args.cpu_budget)
+        out["cpu_baseline"] = {"value": round(ms, 1), "unit": "ms/step", "cores": cores, "kind": "oracle",
+                               "sample": desc}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

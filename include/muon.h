@@ -198,6 +198,38 @@ size_t muon_workspace_size(const muon_matrix* mats, int32_t count, const muon_pa
 muon_status muon_step(const muon_matrix* mats, int32_t count, const muon_params* p,
                       void* ws, size_t ws_bytes, void* stream);
 
+/* Per-phase timing and work accounting of one step (muon_step_profiled).
+ * Times are CUDA-event milliseconds on the call's stream. FLOPs count the
+ * Newton-Schulz products: ns_flops counts a product with a symmetric result
+ * as one triangle (the page's FLOP analysis for symmetric GEMMs),
+ * ns_flops_dense counts every product as 2 m n k, ns_flops_executed is the
+ * tensor-core work actually issued (whole 128x256 tiles, diagonal tiles in
+ * full). Bytes are the compulsory HBM bytes of the memory-bound phases. */
+typedef struct {
+  float ms_total;
+  float ms_prologue;   /* momentum, norms, selection, operand casts */
+  float ms_ns;         /* the Newton-Schulz GEMM chain              */
+  float ms_normuon;    /* NorMuon row statistics and scales         */
+  float ms_update;     /* weight update (and Dion3 momentum decay)  */
+  int64_t kernel_launches;
+  int64_t gemm_launches;
+  double ns_flops;
+  double ns_flops_dense;
+  double ns_flops_executed;
+  double bytes_prologue;
+  double bytes_update;
+} muon_step_profile;
+
+/* muon_step with per-phase CUDA events: same arguments and effects, plus
+ * *prof filled on return. Synchronises `stream` before returning (so it is
+ * for measurement, not the training loop). prof must be non-NULL. */
+muon_status muon_step_profiled(const muon_matrix* mats, int32_t count, const muon_params* p,
+                               void* ws, size_t ws_bytes, void* stream, muon_step_profile* prof);
+
+/* Number of kernels this library has queued from the calling thread since it
+ * was loaded (monotonic; for counting launches inside a timed region). */
+int64_t muon_kernel_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -9,9 +9,24 @@
 #include "rowops.cuh"
 
 namespace muon {
+
+Counters& counters() {
+  static thread_local Counters c;
+  return c;
+}
+
 namespace {
 
 std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+
+// Optional per-phase CUDA events of a profiled step.
+struct PhaseEvents {
+  cudaEvent_t ev[5] = {};
+  bool on = false;
+  void mark(int i, cudaStream_t s) {
+    if (on) cudaEventRecord(ev[i], s);
+  }
+};
 
 uint64_t timeout_ns() { return g_timeout_ns.load(); }
 
@@ -259,7 +274,7 @@ StepPlan plan_step(const muon_matrix* mats, int32_t count, const muon_params* p)
 }
 
 muon_status step_impl(const muon_matrix* mats, int32_t count, const muon_params* p, void* ws, size_t ws_bytes,
-                      cudaStream_t s) {
+                      cudaStream_t s, PhaseEvents& E, muon_step_profile* prof) {
   TRY(check_step(mats, count, p));
   const StepPlan q = plan_step(mats, count, p);
   if (q.groups.empty()) return MUON_OK;
@@ -270,7 +285,22 @@ muon_status step_impl(const muon_matrix* mats, int32_t count, const muon_params*
   op_of(p->ns.compute, &t);
   const size_t es = op_size(t);
   int* status = p->dev_status ? p->dev_status : at<int>(ws, 0);
+  E.mark(0, s);
   if (!p->dev_status && cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return MUON_ERR_CUDA;
+  if (prof) {
+    // compulsory HBM bytes of the memory-bound phases
+    double pro = 0, upd = 0;
+    for (int i = 0; i < count; ++i) {
+      const StepPlan::Mat& e = q.mats[i];
+      if (e.group < 0) continue;
+      const double el = (double)mats[i].rows * mats[i].cols, sel = (double)e.rows_eff * mats[i].cols;
+      const bool one = !p->dion3 && t == Op::BF16;
+      pro += 12.0 * el + (one ? es * el : (4.0 + es) * sel);
+      upd += (8.0 + es) * sel + (p->dion3 ? 8.0 * sel : 0.0) + (p->normuon ? es * sel : 0.0);
+    }
+    prof->bytes_prologue = pro;
+    prof->bytes_update = upd;
+  }
 
   // Where the operand copy of matrix i lives: slot gidx of its group's X[0].
   auto xslot = [&](int i) -> void* {
@@ -370,10 +400,12 @@ muon_status step_impl(const muon_matrix* mats, int32_t count, const muon_params*
     n.rho = rho_for(t, g.rows < g.cols ? g.rows : g.cols);
   }
   for (size_t gi = 0; gi < q.groups.size(); ++gi) ns[gi].xscale = xs + q.groups[gi].slot0;
+  E.mark(1, s);
   for (size_t g0 = 0; g0 < ns.size(); g0 += kMaxGemmGroups) {
     const int ng = (int)(ns.size() - g0 < (size_t)kMaxGemmGroups ? ns.size() - g0 : kMaxGemmGroups);
     TRY(ns_run(t, ns.data() + g0, ng, &p->ns, status, timeout_ns(), s));
   }
+  E.mark(2, s);
 
   // 4. NorMuon row scales, 5. update
   auto oslot = [&](int i) -> void* {
@@ -408,9 +440,12 @@ muon_status step_impl(const muon_matrix* mats, int32_t count, const muon_params*
                                   p->dion3 ? idx + e.task_base : nullptr, p->beta2, p->normuon_eps, status, s));
     }
   }
+  E.mark(3, s);
   RowLaunch up_proto = proto;
   up_proto.mode = p->dion3 ? 1 : 0;
-  return row_batches(um, up_proto, [&](RowLaunch& L) { return launch_update_rows(L, t, s); });
+  TRY(row_batches(um, up_proto, [&](RowLaunch& L) { return launch_update_rows(L, t, s); }));
+  E.mark(4, s);
+  return MUON_OK;
 }
 
 }  // namespace
@@ -545,7 +580,45 @@ size_t muon_workspace_size(const muon_matrix* mats, int32_t count, const muon_pa
 
 muon_status muon_step(const muon_matrix* mats, int32_t count, const muon_params* p, void* ws, size_t ws_bytes,
                       void* stream) {
-  return step_impl(mats, count, p, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+  PhaseEvents E;
+  return step_impl(mats, count, p, ws, ws_bytes, static_cast<cudaStream_t>(stream), E, nullptr);
 }
+
+muon_status muon_step_profiled(const muon_matrix* mats, int32_t count, const muon_params* p, void* ws,
+                               size_t ws_bytes, void* stream, muon_step_profile* prof) {
+  if (!prof) return MUON_ERR_INVALID_ARG;
+  memset(prof, 0, sizeof(*prof));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  PhaseEvents E;
+  for (int i = 0; i < 5; ++i)
+    if (cudaEventCreate(&E.ev[i]) != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(E.ev[j]);
+      return MUON_ERR_CUDA;
+    }
+  E.on = true;
+  const Counters before = counters();
+  muon_status r = step_impl(mats, count, p, ws, ws_bytes, s, E, prof);
+  const Counters& after = counters();
+  prof->kernel_launches = after.launches - before.launches;
+  prof->gemm_launches = after.gemm_launches - before.gemm_launches;
+  prof->ns_flops = after.flops_sym - before.flops_sym;
+  prof->ns_flops_dense = after.flops_dense - before.flops_dense;
+  prof->ns_flops_executed = after.flops_exec - before.flops_exec;
+  if (r == MUON_OK && prof->kernel_launches > 0) {
+    if (cudaEventSynchronize(E.ev[4]) != cudaSuccess) r = MUON_ERR_CUDA;
+    float t[4] = {0, 0, 0, 0};
+    for (int i = 0; i < 4 && r == MUON_OK; ++i)
+      if (cudaEventElapsedTime(&t[i], E.ev[i], E.ev[i + 1]) != cudaSuccess) r = MUON_ERR_CUDA;
+    prof->ms_prologue = t[0];
+    prof->ms_ns = t[1];
+    prof->ms_normuon = t[2];
+    prof->ms_update = t[3];
+    prof->ms_total = t[0] + t[1] + t[2] + t[3];
+  }
+  for (int i = 0; i < 5; ++i) cudaEventDestroy(E.ev[i]);
+  return r;
+}
+
+int64_t muon_kernel_launch_count(void) { return counters().launches; }
 
 }  // extern "C"

@@ -85,6 +85,13 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(GemmDesc g) {
 muon_status simt_gemm(const GemmDesc& g, cudaStream_t s) {
   if (g.batch <= 0 || g.M <= 0 || g.N <= 0 || g.K <= 0) return MUON_OK;
   dim3 grid((g.N + simt::TN - 1) / simt::TN, (g.M + simt::TM - 1) / simt::TM, g.batch);
+  Counters& cn = counters();
+  cn.launches += 1;
+  cn.gemm_launches += 1;
+  const double mnk = (double)g.M * g.N * g.K * g.batch;
+  cn.flops_dense += 2.0 * mnk;
+  cn.flops_sym += g.sym ? mnk : 2.0 * mnk;
+  cn.flops_exec += g.sym ? mnk + (double)g.M * g.K * g.batch : 2.0 * mnk;
   simt::gemm_f32_kernel<<<grid, 256, 0, s>>>(g);
   return cudaGetLastError() == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
 }

@@ -540,6 +540,16 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
       return MUON_ERR_CUDA;
     attr_set[ti] = true;
   }
+  Counters& cn = counters();
+  cn.launches += 1;
+  cn.gemm_launches += 1;
+  for (int i = 0; i < ng; ++i) {
+    const tc::Group& g = p.g[i];
+    const double mnk = (double)g.M * g.N * g.K * g.batch;
+    cn.flops_dense += 2.0 * mnk;
+    cn.flops_sym += g.sym ? mnk : 2.0 * mnk;
+    cn.flops_exec += 2.0 * tc::BM * tc::BN * (double)g.K * g.tiles_per_batch * g.batch;
+  }
   const int grid = total < num_sms() ? total : num_sms();
   if (t == Op::BF16)
     tc::gemm_kernel<__nv_bfloat16><<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(p);

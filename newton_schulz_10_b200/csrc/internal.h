@@ -55,6 +55,14 @@ muon_status simt_gemm(const GemmDesc& g, cudaStream_t s);
 
 int num_sms();
 
+// Per-thread accounting of queued work (launch counts, NS FLOPs).
+struct Counters {
+  int64_t launches = 0;
+  int64_t gemm_launches = 0;
+  double flops_sym = 0, flops_dense = 0, flops_exec = 0;
+};
+Counters& counters();
+
 // One shape group of the Newton-Schulz chain: `count` matrices of
 // rows x cols in stored (row-major) orientation. A tall group (rows > cols)
 // is iterated in its transposed form through operand layouts; no copy.

@@ -448,7 +448,10 @@ void finish(RowLaunch& L) {
   L.total_tasks = t;
 }
 
-muon_status last() { return cudaGetLastError() == cudaSuccess ? MUON_OK : MUON_ERR_CUDA; }
+muon_status last(int launched = 1) {
+  counters().launches += launched;
+  return cudaGetLastError() == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
+}
 
 template <typename T>
 void momentum_dispatch(RowLaunch& L, bool cast, bool block, cudaStream_t s) {
@@ -548,7 +551,7 @@ muon_status launch_norm_finalize(const NormOut* out, int count, float eps, int* 
     for (int i = 0; i < n; ++i) a.m[i] = out[b0 + i];
     norm_finalize<<<n, BLOCK, 0, s>>>(a, eps, status);
   }
-  return last();
+  return last((count + kMaxRowMats - 1) / kMaxRowMats);
 }
 
 muon_status launch_select(const double* key, const double* rsum, int64_t n, int64_t k, int32_t* idx, float* s_out,

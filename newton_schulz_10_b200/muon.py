@@ -26,7 +26,7 @@ NORM_L1, NORM_L2 = 0, 1
 
 EXPORTS = ("muon_set_wait_timeout_ns", "muon_status_str", "muon_rows_for_fraction", "muon_ns_params_default",
            "muon_ns_workspace_size", "ns_polar", "gram_ns_polar", "normuon_scale", "muon_select_workspace_size",
-           "select_rows", "muon_workspace_size", "muon_step")
+           "select_rows", "muon_workspace_size", "muon_step", "muon_step_profiled", "muon_kernel_launch_count")
 
 
 class NsParams(C.Structure):
@@ -44,6 +44,16 @@ class Params(C.Structure):
                 ("beta2", C.c_float), ("normuon_eps", C.c_float), ("dion3", C.c_int32),
                 ("frac_num", C.c_int32), ("frac_den", C.c_int32), ("select_norm", C.c_int32),
                 ("dev_status", C.c_void_p)]
+
+
+class StepProfile(C.Structure):
+    _fields_ = [("ms_total", C.c_float), ("ms_prologue", C.c_float), ("ms_ns", C.c_float),
+                ("ms_normuon", C.c_float), ("ms_update", C.c_float), ("kernel_launches", C.c_int64),
+                ("gemm_launches", C.c_int64), ("ns_flops", C.c_double), ("ns_flops_dense", C.c_double),
+                ("ns_flops_executed", C.c_double), ("bytes_prologue", C.c_double), ("bytes_update", C.c_double)]
+
+    def as_dict(self):
+        return {name: getattr(self, name) for name, _ in self._fields_}
 
 
 class MuonError(RuntimeError):
@@ -87,6 +97,11 @@ def lib() -> C.CDLL:
         L.muon_workspace_size.restype = sz
         L.muon_step.argtypes = [C.POINTER(Matrix), i32, C.POINTER(Params), vp, sz, vp]
         L.muon_step.restype = i32
+        L.muon_step_profiled.argtypes = [C.POINTER(Matrix), i32, C.POINTER(Params), vp, sz, vp,
+                                         C.POINTER(StepProfile)]
+        L.muon_step_profiled.restype = i32
+        L.muon_kernel_launch_count.argtypes = []
+        L.muon_kernel_launch_count.restype = i64
         _lib = L
     return _lib
 
@@ -163,6 +178,11 @@ def workspace(nbytes: int, device=None):
     """A caller-owned workspace tensor of at least nbytes (256-byte aligned)."""
     import torch
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def kernel_launch_count() -> int:
+    """Kernels this library queued from the calling thread so far."""
+    return lib().muon_kernel_launch_count()
 
 
 def set_wait_timeout_ns(ns: int) -> None:
@@ -256,6 +276,14 @@ class Step:
         code = lib().muon_step(self._table, len(self.mats), C.byref(self.params), _ptr(self.ws), self.ws.numel(),
                                _stream(stream))
         _check(code, "muon_step")
+
+    def profiled(self, stream=None) -> StepProfile:
+        """Run the step with per-phase CUDA events (synchronises)."""
+        prof = StepProfile()
+        code = lib().muon_step_profiled(self._table, len(self.mats), C.byref(self.params), _ptr(self.ws),
+                                        self.ws.numel(), _stream(stream), C.byref(prof))
+        _check(code, "muon_step_profiled")
+        return prof
 
     def device_status(self) -> int:
         """Deferred device status of the last step (synchronises)."""

@@ -69,6 +69,9 @@ def test_ns_polar_bf16_input_output():
 @pytest.mark.parametrize("restart", [3, 0])
 @pytest.mark.parametrize("shape", [(256, 1024), (200, 520), (520, 200), (96, 96)])
 def test_gram_ns_polar(compute, restart, shape):
+    if compute == mu.BF16 and shape[0] == shape[1]:
+        pytest.skip("bf16 Gram on a square Gaussian input exceeds 2e-2 by the algorithm itself "
+                    "(see test_gram_bf16_square_matches_emulation)")
     X = gauss(shape, 300 + shape[0])
     p = mu.ns_params(gram=True, restart_at=restart, compute=compute)
     Og, ws = mu.gram_ns_polar(dev(X), p, out_dtype=torch.float32)
@@ -78,17 +81,71 @@ def test_gram_ns_polar(compute, restart, shape):
     assert rel(host(Og), want) < (TOL32 if compute == mu.F32 else TOL16)
 
 
-@pytest.mark.parametrize("gram", [False, True])
-def test_spectrum_matrix(gram):
-    """Singular values log-uniform in [1e-4, 1] (the spectrum workload, small)."""
+def _emulate_bf16(x, role):
+    return bf16_values(np.asarray(x, np.float32))
+
+
+@pytest.mark.parametrize("restart", [3, 0])
+def test_gram_bf16_square_matches_emulation(restart):
+    """A square Gaussian matrix has singular values down to ~0, where T = 5
+    steps amplify rounding ~a^5 = 489 times. In bf16 the Gram iteration then
+    misses the exact polar factor by more than 2e-2 by the algorithm itself:
+    the oracle, rounding to bf16 at the same storage points, misses it by the
+    same amount. The GPU result must not be worse than that emulation by more
+    than 25%."""
+    X = gauss((96, 96), 396)
+    exact = O.gram_newton_schulz(X.astype(np.float64), COEFFS5, restart_at=restart)
+    emul = O.gram_newton_schulz(X.astype(np.float64), COEFFS5, restart_at=restart, store=_emulate_bf16)
+    Og, ws = mu.gram_ns_polar(dev(X), mu.ns_params(gram=True, restart_at=restart, compute=mu.BF16),
+                              out_dtype=torch.float32)
+    assert status_of(ws) == mu.OK
+    e_alg = rel(emul, exact)
+    assert e_alg > 2e-2
+    assert rel(host(Og), exact) < 1.25 * e_alg
+
+
+def _emulate_f16(n):
+    """fp16 storage as the library stores it: X as sqrt(n) X, R as n R."""
+    kappa, rho = np.sqrt(n), float(n)
+
+    def store(x, role):
+        x = np.asarray(x, np.float64)
+        if role in ("X0", "X"):
+            return (x * kappa).astype(np.float16).astype(np.float64) / kappa
+        if role in ("R", "ZR"):
+            return (x * rho).astype(np.float16).astype(np.float64) / rho
+        return x.astype(np.float16).astype(np.float64)
+    return store
+
+
+@pytest.mark.parametrize("gram,compute", [(False, mu.F16), (False, mu.BF16), (True, mu.F16)])
+def test_spectrum_matrix(gram, compute):
+    """Singular values log-uniform in [1e-4, 1] (the spectrum workload,
+    256 x 1024). After normalisation the smallest are ~1e-5, where T = 5
+    quintic steps amplify any rounding ~a^5 = 489 times; how far a half
+    precision chain lands from the exact polar factor is then set by the
+    arithmetic, not by the kernels. Checks: (1) on the well-conditioned
+    directions (normalised sigma > 1e-2) the error is < 2e-2; (2) overall the
+    GPU is within 25% of the oracle run with the same half-precision storage;
+    (3) where that emulated algorithm meets 2e-2 (fp16 standard), the GPU
+    meets 2e-2 too."""
     X, _ = inputs.spectrum_matrix(256, 1024, -4.0, seed=31)
     X32 = X.astype(np.float32)
-    p = mu.ns_params(gram=gram, compute=mu.F16 if gram else mu.BF16)
+    p = mu.ns_params(gram=gram, compute=compute)
     Og, ws = mu.ns_polar(dev(X32, torch.bfloat16), p, out_dtype=torch.float32)
     assert status_of(ws) == mu.OK
     Xb = bf16_values(X32)
-    want = O.newton_schulz(Xb, COEFFS5)
-    assert rel(host(Og), want) < TOL16
+    exact = O.newton_schulz(Xb, COEFFS5)
+    store = _emulate_f16(256) if compute == mu.F16 else _emulate_bf16
+    emul = (O.gram_newton_schulz(Xb, COEFFS5, store=store) if gram else O.newton_schulz(Xb, COEFFS5, store=store))
+    got = host(Og)
+    U, s, _ = np.linalg.svd(Xb, full_matrices=False)
+    well = (s / np.linalg.norm(s)) > 1e-2
+    assert np.linalg.norm((U.T @ (got - exact))[well]) / np.linalg.norm(exact) < TOL16
+    e_alg = rel(emul, exact)
+    assert rel(got, exact) < 1.25 * max(e_alg, 4e-3)
+    if e_alg < TOL16:
+        assert rel(got, exact) < TOL16
 
 
 def test_time_varying_coefficients():
@@ -189,11 +246,14 @@ def test_step_fp32_single():
 
 
 MIXED = [(128, 128), (128, 128), (128, 384), (384, 128), (100, 260), (260, 100), (64, 64)]
+MIXED_RECT = [(128, 384), (128, 384), (384, 128), (100, 260), (260, 100), (64, 640)]
 
 
 @pytest.mark.parametrize("gram,compute", [(False, mu.BF16), (True, mu.F16), (True, mu.BF16), (False, mu.F32)])
 def test_step_batched(gram, compute):
-    state = make_state(MIXED, 2000, m_std=2e-3)
+    # bf16 Gram only on rectangular matrices (square ones: see test_gram_bf16_square_matches_emulation)
+    shapes = MIXED_RECT if (gram and compute == mu.BF16) else MIXED
+    state = make_state(shapes, 2000, m_std=2e-3)
     p = mu.step_params(ns=mu.ns_params(gram=gram, compute=compute))
     got, st = run_step(state, p)
     assert st == mu.OK
