@@ -186,6 +186,24 @@ size_t muon_select_workspace_size(int64_t n);
 muon_status select_rows(const float* M, int64_t n, int64_t m, int64_t k, muon_norm norm,
                         int32_t* idx_out, void* ws, size_t ws_bytes, void* stream);
 
+/* select_rows without a workspace, for callers that cannot allocate device
+ * memory when they need a selection (a pool that is already carved up, a
+ * runtime that forbids cudaMalloc after start-up because it can synchronise
+ * the device, a C host without an allocator). The page has no counterpart:
+ * this is a packaging of select_rows, same arguments and same result,
+ * minus the workspace, plus an optional dev_status for deferred errors.
+ *
+ * Scratch: a fixed 1 MiB + 256 B __device__ array inside libmuon.so, held by
+ * every GPU that loads the library until the process exits. n is limited to
+ * 65536 rows (MUON_ERR_SHAPE beyond). The first call on each device looks up
+ * the array's device address (cudaGetSymbolAddress) with that device
+ * current; make that first call before any stream capture. All calls share
+ * the one array: calls whose work overlaps on the GPU (different streams, or
+ * different host threads, without ordering between them) race and give
+ * wrong indices; calls ordered on one stream are safe. Allocates nothing. */
+muon_status select_rows_noalloc(const float* M, int64_t n, int64_t m, int64_t k, muon_norm norm,
+                                int32_t* idx_out, int32_t* dev_status, void* stream);
+
 /* Workspace bytes for muon_step over mats[0..count) with parameters p
  * (0 for invalid arguments). */
 size_t muon_workspace_size(const muon_matrix* mats, int32_t count, const muon_params* p);

@@ -26,7 +26,8 @@ NORM_L1, NORM_L2 = 0, 1
 
 EXPORTS = ("muon_set_wait_timeout_ns", "muon_status_str", "muon_rows_for_fraction", "muon_ns_params_default",
            "muon_ns_workspace_size", "ns_polar", "gram_ns_polar", "normuon_scale", "muon_select_workspace_size",
-           "select_rows", "muon_workspace_size", "muon_step", "muon_step_profiled", "muon_kernel_launch_count")
+           "select_rows", "muon_workspace_size", "muon_step", "muon_step_profiled", "muon_kernel_launch_count",
+           "select_rows_noalloc")
 
 
 class NsParams(C.Structure):
@@ -93,6 +94,8 @@ def lib() -> C.CDLL:
         L.muon_select_workspace_size.restype = sz
         L.select_rows.argtypes = [vp, i64, i64, i64, i32, vp, vp, sz, vp]
         L.select_rows.restype = i32
+        L.select_rows_noalloc.argtypes = [vp, i64, i64, i64, i32, vp, vp, vp]
+        L.select_rows_noalloc.restype = i32
         L.muon_workspace_size.argtypes = [C.POINTER(Matrix), i32, C.POINTER(Params)]
         L.muon_workspace_size.restype = sz
         L.muon_step.argtypes = [C.POINTER(Matrix), i32, C.POINTER(Params), vp, sz, vp]
@@ -238,6 +241,19 @@ def select_rows(M, k: int, norm: int = NORM_L1, ws=None, stream=None):
         ws = workspace(lib().muon_select_workspace_size(n), M.device)
     code = lib().select_rows(_ptr(M), n, m, k, norm, _ptr(idx), _ptr(ws), ws.numel(), _stream(stream))
     _check(code, "select_rows")
+    return idx
+
+
+def select_rows_noalloc(M, k: int, norm: int = NORM_L1, idx=None, dev_status=None, stream=None):
+    """select_rows without a workspace (fixed scratch inside the library; at
+    most 65536 rows; calls that overlap on the GPU race). idx may be passed
+    in to avoid allocating the output here too."""
+    import torch
+    n, m = M.shape
+    if idx is None:
+        idx = torch.empty(k, dtype=torch.int32, device=M.device)
+    code = lib().select_rows_noalloc(_ptr(M), n, m, k, norm, _ptr(idx), _ptr(dev_status), _stream(stream))
+    _check(code, "select_rows_noalloc")
     return idx
 
 
