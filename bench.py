@@ -219,6 +219,17 @@ def run_ours(args, rank, world, local_rank):
         step(stream)
     torch.cuda.synchronize()
     status = step.device_status()
+    run = step
+    graph = None
+    if args.graph:
+        # capture one whole step (all its launches) in a CUDA graph, replay it
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step(torch.cuda.current_stream())
+        run = lambda s=None: graph.replay()  # noqa: E731
+        for _ in range(2):
+            run()
+        torch.cuda.synchronize()
 
     # --- device-resident timing -------------------------------------------
     if world > 1:
@@ -230,11 +241,13 @@ def run_ours(args, rank, world, local_rank):
         t0 = time.time()
         e0.record(stream)
         for _ in range(args.steps):
-            step(stream)
+            run(stream)
         e1.record(stream)
         torch.cuda.synchronize()
         t1 = time.time()
     launches = mu.kernel_launch_count() - n0
+    if graph is not None:  # replays queue no launches from the host: count the captured ones
+        launches = args.steps * step.profiled(stream).kernel_launches
     if world > 1:
         dist.barrier()
     ms = e0.elapsed_time(e1) / args.steps
@@ -270,7 +283,7 @@ def run_ours(args, rank, world, local_rank):
     for _ in range(e2e_steps):
         for hg, (_, _, G, _) in zip(hostG, state):
             G.copy_(hg, non_blocking=True)
-        step(stream)
+        run(stream)
         for hw, (W, _, _, _) in zip(hostW, state):
             hw.copy_(W, non_blocking=True)
     f1.record(stream)
@@ -307,6 +320,7 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": cfg["compute"], "data": "synthetic",
         "config": {"workload": args.workload, "description": cfg["desc"], "matrices": len(specs),
+                   "cuda_graph": bool(args.graph),
                    "elements": elems, "state_bytes": 12 * elems,
                    "l2": "inputs larger than L2 (fp32 W, M, G resident in HBM)",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
@@ -317,6 +331,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches,
         "clocks": clocks,
         "device_status": mu.status_str(status),
+        "cuda_graph": bool(args.graph),
     }
     return out
 
@@ -491,6 +506,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt124m")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", type=int, default=1, help="1: replay the step as one captured CUDA graph")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

@@ -433,12 +433,14 @@ muon_status step_impl(const muon_matrix* mats, int32_t count, const muon_params*
   }
   if (p->normuon) {
     TRY(row_batches(um, proto, [&](RowLaunch& L) { return launch_normuon_rows(L, t, s); }));
+    std::vector<NormuonMat> nm;
     for (int i = 0; i < count; ++i) {
       const StepPlan::Mat& e = q.mats[i];
       if (e.group < 0) continue;
-      TRY(launch_normuon_finalize(rscale + e.task_base, e.rows_eff, mats[i].cols, mats[i].v,
-                                  p->dion3 ? idx + e.task_base : nullptr, p->beta2, p->normuon_eps, status, s));
+      nm.push_back(NormuonMat{rscale + e.task_base, e.rows_eff, mats[i].cols, mats[i].v,
+                              p->dion3 ? idx + e.task_base : nullptr});
     }
+    TRY(launch_normuon_finalize_batched(nm.data(), (int)nm.size(), p->beta2, p->normuon_eps, status, s));
   }
   E.mark(3, s);
   RowLaunch up_proto = proto;

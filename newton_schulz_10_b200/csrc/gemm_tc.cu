@@ -1,6 +1,6 @@
 // Tensor-core GEMM for the Newton-Schulz chain on sm_100a.
 //
-// Persistent, warp-specialised kernel: one CTA per SM, 256 threads.
+// Persistent, warp-specialised kernel: one CTA per SM, 384 threads.
 //   warp 0      TMA producer (one elected thread): A and B tiles into a
 //               4-stage shared-memory ring, 128-byte swizzle, no multicast
 //   warp 1      MMA issuer (one thread): tcgen05.mma kind::f16, 128x256x16
@@ -8,10 +8,15 @@
 //   warp 2      allocates / frees the 512 TMEM columns (two 128x256 fp32
 //               accumulators: the epilogue of tile i overlaps the mainloop of
 //               tile i+1)
-//   warps 4..7  epilogue: tcgen05.ld of 32x32 sub-tiles, fused
-//               alpha*acc + beta*C + gamma*I, narrowing store; for symmetric
-//               outputs the lower-triangle value is also written, transposed
-//               through shared memory, to the mirrored position.
+//   warps 4..11 epilogue, two warps per TMEM lane quarter, each owning 128
+//               of the tile's 256 columns: C rows prefetched into registers,
+//               tcgen05.ld of 32x32 sub-tiles, fused alpha*acc + beta*C +
+//               gamma*I, one rounding to the stored type, then each 32x32
+//               block is staged in 64B-swizzled shared memory and written by
+//               a TMA bulk tensor store (clipped at the matrix edge). For
+//               symmetric outputs a second staged block holds the transpose,
+//               stored at the mirrored position; a block on the diagonal is
+//               symmetrised in shared memory and stored once.
 //
 // Symmetric outputs ("2. Symmetric GEMM Kernels" of the Dion3 page: a
 // triangular scheduler over lower tiles and a transposed-tile epilogue) are
@@ -35,25 +40,30 @@ constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int UMMA_K = 16;
 constexpr int A_STAGE = BM * BK * 2;  // 16 KB
 constexpr int B_STAGE = BN * BK * 2;  // 32 KB
-constexpr int THREADS = 256;
 constexpr int EPI_WARP0 = 4;
+constexpr int EPI_WARPS = 8;                       // two per TMEM lane quarter
+constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
+constexpr int EPI_CHUNKS = BN / 32 / 2;            // 32-column chunks per epilogue warp
 constexpr int TMEM_COLS = 512;
-constexpr int EPI_BUF_WORDS = 32 * 33;  // per epilogue warp (padded 32x32 transpose)
+constexpr int EPI_BLOCK = 32 * 32 * 2;   // one staged 32x32 block of bf16/fp16, 64-byte rows
+constexpr int EPI_BUF = 2 * EPI_BLOCK;    // per epilogue warp: direct block + mirrored block
 // Drains (in-flight copies and MMAs before exit) use their own bound, so that
 // a tiny configurable wait budget never lets a CTA exit with work in flight.
 constexpr uint64_t DRAIN_NS = 1000000000ull;
-constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_STAGE + B_STAGE) + 4 * EPI_BUF_WORDS * 4 +
+constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_STAGE + B_STAGE) + EPI_WARPS * EPI_BUF +
                            (2 * STAGES + 5) * 8 + 16;
+static_assert(SMEM_BYTES <= 232448, "exceeds the opt-in shared memory of one sm_100 CTA");
 
 struct Group {
   CUtensorMap tmA;
   CUtensorMap tmB;
+  CUtensorMap tmD;  // 32x32 boxes, 64-byte swizzle: epilogue stores
   void* D;
   const void* C;
   const float* scale;
   long long ldd, sD, ldc, sC;
   int M, N, K, batch;
-  int a_mn, b_mn, sym, d_f32;
+  int a_mn, b_mn, sym;
   int alpha_pow, beta_pow;
   float alpha, beta, gamma;
   int tiles_m, tiles_n, tiles_per_batch, tile_begin;
@@ -107,40 +117,21 @@ __device__ __forceinline__ float powi(float s, int p) {
   return r;
 }
 
-template <typename T>
-__device__ __forceinline__ void store_row32(const Group& g, const Tile& t, int row, int c0, const float* v,
-                                            bool full_lower, bool any_lower) {
-  // Direct store of D[row, c0..c0+32). For symmetric outputs only elements
-  // with col <= row are written (full_lower: all 32 are).
-  if (row >= g.M || !any_lower) return;
-  if (g.d_f32) {
-    float* d = reinterpret_cast<float*>(g.D) + (long long)t.b * g.sD + (long long)row * g.ldd + c0;
-    if (full_lower) {
-#pragma unroll
-      for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4*>(d + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-    } else {
-      for (int j = 0; j < 32; ++j)
-        if (c0 + j <= row) d[j] = v[j];
-    }
-  } else {
-    T* d = reinterpret_cast<T*>(g.D) + (long long)t.b * g.sD + (long long)row * g.ldd + c0;
-    if (full_lower) {
-#pragma unroll
-      for (int j = 0; j < 32; j += 8) {
-        uint4 u;
-        u.x = Elem<T>::pack2(v[j], v[j + 1]);
-        u.y = Elem<T>::pack2(v[j + 2], v[j + 3]);
-        u.z = Elem<T>::pack2(v[j + 4], v[j + 5]);
-        u.w = Elem<T>::pack2(v[j + 6], v[j + 7]);
-        *reinterpret_cast<uint4*>(d + j) = u;
-      }
-    } else {
-      for (int j = 0; j < 32; ++j)
-        if (c0 + j <= row) d[j] = Elem<T>::from_f(v[j]);
-    }
-  }
+// Byte offset of element (r, c) of a staged 32x32 block with 64-byte rows
+// and the TMA 64-byte swizzle (16-byte chunk index XOR (r / 2) % 4).
+__device__ __forceinline__ uint32_t sw64(int r, int c) {
+  return (uint32_t)(r * 64 + ((((c >> 3) ^ (r >> 1)) & 3) << 4) + ((c & 7) << 1));
 }
+
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 template <typename T>
 __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant__ Params p) {
@@ -148,8 +139,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE;
-  uint32_t* sEpi = reinterpret_cast<uint32_t*>(sB + STAGES * B_STAGE);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + 4 * EPI_BUF_WORDS);
+  uint8_t* sEpi = sB + STAGES * B_STAGE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + EPI_WARPS * EPI_BUF);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
@@ -167,7 +158,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4 * 32);
+      mbar_init(&tempty[b], EPI_WARPS * 32);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -311,8 +302,11 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     // ------------------------------------------------------------------
     // Epilogue
     // ------------------------------------------------------------------
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    uint32_t* buf = sEpi + q * EPI_BUF_WORDS;
+    const int e = warp - EPI_WARP0;
+    const int q = warp & 3;   // TMEM lane quarter this warp may access
+    const int half = e >> 2;  // which 128 of the tile's 256 columns it owns
+    uint8_t* sd = sEpi + e * EPI_BUF;  // staged direct block (1024-byte aligned)
+    uint8_t* sm = sd + EPI_BLOCK;       // staged mirrored block
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
@@ -328,26 +322,40 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       const float beta = g.beta * powi(s, g.beta_pow);
       const int r0 = t.m0 + q * 32;
       const int row = r0 + lane;
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        const int c0 = t.n0 + ch * 32;
+      const int cbase = t.n0 + half * (BN / 2);
+      // The C rows this thread needs, loaded for all its chunks before the
+      // first TMEM read so their latency overlaps instead of adding up.
+      uint4 cv[EPI_CHUNKS][4];
+      const bool want_c = g.beta != 0.f && row < g.M;
+      if (want_c) {
+        const T* c = reinterpret_cast<const T*>(g.C) + (long long)t.b * g.sC + (long long)row * g.ldc + cbase;
+#pragma unroll
+        for (int ch = 0; ch < EPI_CHUNKS; ++ch)
+          if (cbase + ch * 32 < g.N) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) cv[ch][j] = *reinterpret_cast<const uint4*>(c + ch * 32 + j * 8);
+          }
+      }
+#pragma unroll
+      for (int ch = 0; ch < EPI_CHUNKS; ++ch) {
+        const int c0 = cbase + ch * 32;
         if (c0 >= g.N) break;                      // warp-uniform
         if (g.sym && c0 > r0 + 31) break;          // whole sub-tile above the diagonal
         uint32_t raw[32];
-        tmem_ld_32x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + ch * 32, raw);
+        tmem_ld_32x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + half * (BN / 2) + ch * 32, raw);
         tmem_wait_ld();
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = alpha * __uint_as_float(raw[j]);
-        if (g.beta != 0.f && row < g.M) {
-          const T* c = reinterpret_cast<const T*>(g.C) + (long long)t.b * g.sC + (long long)row * g.ldc + c0;
+        if (want_c) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            const uint4 u = *reinterpret_cast<const uint4*>(c + j);
+          for (int j = 0; j < 4; ++j) {
+            const uint4 u = cv[ch][j];
             float2 f;
-            f = Elem<T>::unpack2(u.x); v[j] += beta * f.x; v[j + 1] += beta * f.y;
-            f = Elem<T>::unpack2(u.y); v[j + 2] += beta * f.x; v[j + 3] += beta * f.y;
-            f = Elem<T>::unpack2(u.z); v[j + 4] += beta * f.x; v[j + 5] += beta * f.y;
-            f = Elem<T>::unpack2(u.w); v[j + 6] += beta * f.x; v[j + 7] += beta * f.y;
+            f = Elem<T>::unpack2(u.x); v[8 * j] += beta * f.x; v[8 * j + 1] += beta * f.y;
+            f = Elem<T>::unpack2(u.y); v[8 * j + 2] += beta * f.x; v[8 * j + 3] += beta * f.y;
+            f = Elem<T>::unpack2(u.z); v[8 * j + 4] += beta * f.x; v[8 * j + 5] += beta * f.y;
+            f = Elem<T>::unpack2(u.w); v[8 * j + 6] += beta * f.x; v[8 * j + 7] += beta * f.y;
           }
         }
         if (g.gamma != 0.f) {
@@ -358,53 +366,39 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
               if (jj == j) v[jj] += g.gamma;
           }
         }
-        // round once to the stored type so the mirror holds identical values
-        if (!g.d_f32) {
+        // Round once to the stored type: the direct and mirrored copies of an
+        // element are the same bits, so D is exactly symmetric.
+        uint32_t pk[16];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = Elem<T>::to_f(Elem<T>::from_f(v[j]));
+        for (int j = 0; j < 16; ++j) pk[j] = Elem<T>::pack2(v[2 * j], v[2 * j + 1]);
+        const bool diag = g.sym && c0 == r0;   // the block straddles the diagonal
+        const bool mirror = g.sym && r0 > c0;  // strictly lower: also store its transpose
+        // the previous chunk's bulk stores must have finished reading the staging blocks
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<uint4*>(sd + sw64(lane, 8 * k)) =
+              make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        if (diag) {
+          // symmetrise the diagonal block: above the diagonal (row j < col)
+          // takes the value computed below it, D[j][lane] = D[lane][j]
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (j < lane) *reinterpret_cast<uint16_t*>(sd + sw64(j, lane)) = (uint16_t)(pk[j >> 1] >> ((j & 1) * 16));
         }
-        const bool full_lower = !g.sym || (c0 + 31 <= row);
-        const bool any_lower = !g.sym || (c0 <= row);
-        store_row32<T>(g, t, row, c0, v, full_lower, any_lower);
-        if (g.sym && r0 + 31 > c0) {
-          // mirror: D[c, r] = D[r, c] for r > c, via a 32x32 transpose
+        if (mirror) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) buf[lane * 33 + j] = __float_as_uint(v[j]);
-          __syncwarp();
-          const int c = c0 + lane;  // mirrored row
-          if (c < g.N) {
-            float w[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) w[i] = __uint_as_float(buf[i * 33 + lane]);
-            const bool all = (r0 > c) && (r0 + 31 < g.M);
-            if (g.d_f32) {
-              float* d = reinterpret_cast<float*>(g.D) + (long long)t.b * g.sD + (long long)c * g.ldd + r0;
-              if (all) {
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(d + i) = make_float4(w[i], w[i + 1], w[i + 2], w[i + 3]);
-              } else {
-                for (int i = 0; i < 32; ++i)
-                  if (r0 + i > c && r0 + i < g.M) d[i] = w[i];
-              }
-            } else {
-              T* d = reinterpret_cast<T*>(g.D) + (long long)t.b * g.sD + (long long)c * g.ldd + r0;
-              if (all) {
-#pragma unroll
-                for (int i = 0; i < 32; i += 8) {
-                  uint4 u;
-                  u.x = Elem<T>::pack2(w[i], w[i + 1]);
-                  u.y = Elem<T>::pack2(w[i + 2], w[i + 3]);
-                  u.z = Elem<T>::pack2(w[i + 4], w[i + 5]);
-                  u.w = Elem<T>::pack2(w[i + 6], w[i + 7]);
-                  *reinterpret_cast<uint4*>(d + i) = u;
-                }
-              } else {
-                for (int i = 0; i < 32; ++i)
-                  if (r0 + i > c && r0 + i < g.M) d[i] = Elem<T>::from_f(w[i]);
-              }
-            }
-          }
-          __syncwarp();
+          for (int j = 0; j < 32; ++j)
+            *reinterpret_cast<uint16_t*>(sm + sw64(j, lane)) = (uint16_t)(pk[j >> 1] >> ((j & 1) * 16));
+        }
+        fence_async_smem();  // generic-proxy writes become visible to the bulk copy
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&g.tmD, smem_u32(sd), c0, r0, t.b);
+          if (mirror) tma_store_3d(&g.tmD, smem_u32(sm), r0, c0, t.b);
+          bulk_commit();
         }
       }
       tc_fence_before();
@@ -414,6 +408,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         acc_phase ^= 1;
       }
     }
+    if (lane == 0) bulk_wait0();  // every staged block written before the CTA exits
   }
 
   tc_fence_before();
@@ -448,18 +443,20 @@ EncodeTiledFn encode_fn() {
 }
 
 // 3-D map over [batch][outer][inner] with row stride ld and batch stride
-// (elements), box {64, box_outer, 1}, 128-byte swizzle, zero fill out of range.
+// (elements), box {box_inner, box_outer, 1}, zero fill out of range (loads)
+// and clipping (stores).
 bool make_map(CUtensorMap* m, Op t, const void* base, int64_t inner, int64_t outer, int64_t batch, int64_t ld,
-              int64_t bstride, int box_outer) {
+              int64_t bstride, int box_outer, int box_inner = 64,
+              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const CUtensorMapDataType dt = t == Op::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)outer, (cuuint64_t)batch};
   cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)(batch > 1 ? bstride : ld * outer) * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)box_outer, 1};
+  cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -492,6 +489,7 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
                      : make_map(&g.tmA, t, d.A, d.K, d.M, d.batch, d.lda, d.strideA, tc::BM);
     ok = ok && (d.b_mn ? make_map(&g.tmB, t, d.B, d.N, d.K, d.batch, d.ldb, d.strideB, 64)
                        : make_map(&g.tmB, t, d.B, d.K, d.N, d.batch, d.ldb, d.strideB, tc::BN));
+    ok = ok && make_map(&g.tmD, t, d.D, d.N, d.M, d.batch, d.ldd, d.strideD, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
     if (!ok) return MUON_ERR_CUDA;
     g.D = d.D;
     g.C = d.C;
@@ -507,7 +505,6 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
     g.a_mn = d.a_mn;
     g.b_mn = d.b_mn;
     g.sym = d.sym;
-    g.d_f32 = d.d_f32;
     g.alpha_pow = d.alpha_pow;
     g.beta_pow = d.beta_pow;
     g.alpha = d.alpha;

@@ -43,7 +43,6 @@ struct GemmDesc {
   float alpha, beta, gamma;
   const float* scale;
   int alpha_pow, beta_pow;
-  int d_f32;  // tensor-core path only: write D as fp32 instead of the operand type
 };
 
 // Tensor-core GEMM (tcgen05 + TMEM + TMA), all groups in one persistent launch.

@@ -390,9 +390,31 @@ __global__ void __launch_bounds__(SEL_THREADS) select_topk(const double* key, co
   }
 }
 
+__device__ void normuon_finalize_block(float* rscale, int64_t k, int64_t m, float* v, const int32_t* idx,
+                                       float beta2, float eps, int* status, double* scratch);
+
 __global__ void __launch_bounds__(BLOCK) normuon_finalize(float* rscale, int64_t k, int64_t m, float* v,
                                                           const int32_t* idx, float beta2, float eps, int* status) {
   __shared__ double scratch[32];
+  normuon_finalize_block(rscale, k, m, v, idx, beta2, eps, status, scratch);
+}
+
+struct NormuonArgs {
+  NormuonMat m[kMaxRowMats];
+};
+
+__global__ void __launch_bounds__(BLOCK) normuon_finalize_many(const __grid_constant__ NormuonArgs a, float beta2,
+                                                               float eps, int* status) {
+  __shared__ double scratch[32];
+  const NormuonMat& o = a.m[blockIdx.x];
+  normuon_finalize_block(o.rscale, o.k, o.m, o.v, o.idx, beta2, eps, status, scratch);
+}
+
+// Eq. (2) for one matrix by one block: v_j <- beta2 v_j + (1 - beta2) r_i / m,
+// d_i = 1 / (sqrt(v_j) + eps), ratio = sqrt(sum r) / sqrt(sum d^2 r),
+// rscale[i] <- ratio * d_i (rscale holds r_i on entry).
+__device__ void normuon_finalize_block(float* rscale, int64_t k, int64_t m, float* v, const int32_t* idx,
+                                       float beta2, float eps, int* status, double* scratch) {
   double sum_r = 0.0, sum_dr = 0.0;
   const float inv_m = 1.f / (float)m;
   for (int64_t i = threadIdx.x; i < k; i += BLOCK) {
@@ -564,6 +586,19 @@ muon_status launch_normuon_finalize(float* rscale, int64_t k, int64_t m, float* 
                                     float eps, int* status, cudaStream_t s) {
   normuon_finalize<<<1, BLOCK, 0, s>>>(rscale, k, m, v, idx, beta2, eps, status);
   return last();
+}
+
+muon_status launch_normuon_finalize_batched(const NormuonMat* mats, int count, float beta2, float eps, int* status,
+                                            cudaStream_t s) {
+  int launched = 0;
+  for (int b0 = 0; b0 < count; b0 += kMaxRowMats) {
+    NormuonArgs a;
+    const int n = count - b0 < kMaxRowMats ? count - b0 : kMaxRowMats;
+    for (int i = 0; i < n; ++i) a.m[i] = mats[b0 + i];
+    normuon_finalize_many<<<n, BLOCK, 0, s>>>(a, beta2, eps, status);
+    ++launched;
+  }
+  return last(launched);
 }
 
 muon_status launch_copy_out(const void* in, Op it, int64_t ldi, void* out, Op ot, int64_t rows, int64_t cols,

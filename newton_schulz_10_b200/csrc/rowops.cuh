@@ -75,6 +75,16 @@ muon_status launch_select(const double* key, const double* rsum, int64_t n, int6
 muon_status launch_normuon_finalize(float* rscale, int64_t k, int64_t m, float* v, const int32_t* idx, float beta2,
                                     float eps, int* status, cudaStream_t s);
 
+// The same for many matrices, one block per matrix, kMaxRowMats per launch.
+struct NormuonMat {
+  float* rscale;
+  int64_t k, m;
+  float* v;
+  const int32_t* idx;
+};
+muon_status launch_normuon_finalize_batched(const NormuonMat* mats, int count, float beta2, float eps, int* status,
+                                            cudaStream_t s);
+
 // Copy an internal (padded) matrix to a caller buffer (ld = cols).
 muon_status launch_copy_out(const void* in, Op it, int64_t ldi, void* out, Op ot, int64_t rows, int64_t cols,
                             cudaStream_t s);

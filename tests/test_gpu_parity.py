@@ -324,3 +324,29 @@ def test_step_deterministic_and_resumable():
     mu.muon_step(d3, p)
     for r, (a, b, _, d) in zip(ref, d3):
         assert np.array_equal(r[0], host(a)) and np.array_equal(r[1], host(b)) and np.array_equal(r[2], host(d))
+
+
+def test_step_cuda_graph_matches_eager():
+    """A step captured in a CUDA graph and replayed gives the same bits as the
+    same step run eagerly (the page captures its step in a graph to remove
+    launch overhead at small scale)."""
+    shapes = [(128, 384), (384, 128), (64, 64)]
+    state = make_state(shapes, 7000, m_std=1e-3)
+    p = mu.step_params(normuon=True)
+    d1 = [(dev(W), dev(M), dev(G), dev(v)) for (W, M, G, v) in state]
+    s1 = mu.Step(d1, p)
+    s1()
+    s1()
+    d2 = [(dev(W), dev(M), dev(G), dev(v)) for (W, M, G, v) in state]
+    s2 = mu.Step(d2, p)
+    s2()  # first step eagerly (also sets kernel attributes before capture)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        s2(torch.cuda.current_stream())
+    graph.replay()
+    torch.cuda.synchronize()
+    assert s2.device_status() == mu.OK
+    for a, b in zip(d1, d2):
+        for x, y in zip(a, b):
+            assert torch.equal(x, y)
