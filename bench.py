@@ -190,6 +190,50 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def end_to_end(args, state, run, stream, elems, big, world):
+    """Same step with host buffers: each step copies that step's gradients
+    from pinned host memory to the device and the updated weights back."""
+    import torch
+    import torch.distributed as dist
+
+    # each step: H2D copy of that step's gradients from pinned memory, the
+    # step, D2H copy of the updated weights into pinned memory
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except ImportError:
+        avail = 1 << 62
+    if 2 * 4 * elems > 0.5 * avail:
+        return {"value": None, "unit": "ms/step", "h2d_bytes_per_step": 4 * elems, "d2h_bytes_per_step": 4 * elems,
+                "reason": f"pinned host buffers need {8 * elems / 1e9:.1f} GB, {avail / 1e9:.1f} GB available"}
+    hostG = [torch.empty_like(G, device="cpu").pin_memory() for (_, _, G, _) in state]
+    hostW = [torch.empty_like(W, device="cpu").pin_memory() for (W, _, _, _) in state]
+    for hg, (_, _, G, _) in zip(hostG, state):
+        hg.copy_(G)
+    e2e_steps = max(1, min(args.steps, 20 if not big else 3))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        for hg, (_, _, G, _) in zip(hostG, state):
+            G.copy_(hg, non_blocking=True)
+        run(stream)
+        for hw, (W, _, _, _) in zip(hostW, state):
+            hw.copy_(W, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1) / e2e_steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    return {"value": round(e2e_ms, 3), "unit": "ms/step", "h2d_bytes_per_step": 4 * elems,
+            "d2h_bytes_per_step": 4 * elems, "what": "G pinned-host->device, step, W device->pinned-host",
+            "steps": e2e_steps}
+
+
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
@@ -261,39 +305,10 @@ def run_ours(args, rank, world, local_rank):
     prof = step.profiled(stream)
 
     # --- end to end through host buffers ------------------------------------
-    # each step: H2D copy of that step's gradients from pinned memory, the
-    # step, D2H copy of the updated weights into pinned memory
-    try:
-        import psutil
-        avail = psutil.virtual_memory().available
-    except ImportError:
-        avail = 1 << 62
-    if 2 * 4 * elems > 0.5 * avail:
-        raise SystemExit("not enough host memory for the end-to-end arm")
-    hostG = [torch.empty_like(G, device="cpu").pin_memory() for (_, _, G, _) in state]
-    hostW = [torch.empty_like(W, device="cpu").pin_memory() for (W, _, _, _) in state]
-    for hg, (_, _, G, _) in zip(hostG, state):
-        hg.copy_(G)
-    e2e_steps = max(1, min(args.steps, 20 if not big else 3))
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(e2e_steps):
-        for hg, (_, _, G, _) in zip(hostG, state):
-            G.copy_(hg, non_blocking=True)
-        run(stream)
-        for hw, (W, _, _, _) in zip(hostW, state):
-            hw.copy_(W, non_blocking=True)
-    f1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1) / e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-
+    if args.no_e2e:
+        e2e = None
+    else:
+        e2e = end_to_end(args, state, run, stream, elems, big, world)
     peaks, peak_kind = measured_peaks()
     long_step = ms > 100.0
     tensor_peak = peaks["bf16_tflops_sustained" if long_step else "bf16_tflops"]
@@ -326,8 +341,7 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "roofline": roof,
         "phases": phases,
-        "e2e": {"value": round(e2e_ms, 3), "unit": "ms/step", "h2d_bytes_per_step": 4 * elems,
-                "d2h_bytes_per_step": 4 * elems, "what": "G pinned-host->device, step, W device->pinned-host"},
+        "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,
         "device_status": mu.status_str(status),
@@ -506,6 +520,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt124m")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end arm")
     ap.add_argument("--graph", type=int, default=1, help="1: replay the step as one captured CUDA graph")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)

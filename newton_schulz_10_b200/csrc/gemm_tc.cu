@@ -36,7 +36,7 @@ namespace muon {
 
 namespace tc {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128, BN = 256, BK = 64;
 constexpr int UMMA_K = 16;
 constexpr int A_STAGE = BM * BK * 2;  // 16 KB
 constexpr int B_STAGE = BN * BK * 2;  // 32 KB
@@ -46,10 +46,11 @@ constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
 constexpr int EPI_CHUNKS = BN / 32 / 2;            // 32-column chunks per epilogue warp
 constexpr int TMEM_COLS = 512;
 constexpr int EPI_BLOCK = 32 * 32 * 2;   // one staged 32x32 block of bf16/fp16, 64-byte rows
-constexpr int EPI_BUF = 2 * EPI_BLOCK;    // per epilogue warp: direct block + mirrored block
 // Drains (in-flight copies and MMAs before exit) use their own bound, so that
 // a tiny configurable wait budget never lets a CTA exit with work in flight.
 constexpr uint64_t DRAIN_NS = 1000000000ull;
+constexpr int STAGES = 4;
+constexpr int EPI_BUF = 2 * EPI_BLOCK;  // per epilogue warp: direct block + mirrored block
 constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_STAGE + B_STAGE) + EPI_WARPS * EPI_BUF +
                            (2 * STAGES + 5) * 8 + 16;
 static_assert(SMEM_BYTES <= 232448, "exceeds the opt-in shared memory of one sm_100 CTA");
@@ -305,8 +306,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     const int e = warp - EPI_WARP0;
     const int q = warp & 3;   // TMEM lane quarter this warp may access
     const int half = e >> 2;  // which 128 of the tile's 256 columns it owns
-    uint8_t* sd = sEpi + e * EPI_BUF;  // staged direct block (1024-byte aligned)
-    uint8_t* sm = sd + EPI_BLOCK;       // staged mirrored block
+    uint8_t* const sd = sEpi + e * EPI_BUF;  // staged direct block (1024-byte aligned)
+    uint8_t* const sm = sd + EPI_BLOCK;       // staged mirrored block
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
@@ -529,14 +530,6 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
   p.status = status;
   p.timeout_ns = timeout_ns;
 
-  static bool attr_set[2] = {false, false};
-  const int ti = t == Op::BF16 ? 0 : 1;
-  const void* fn = t == Op::BF16 ? (const void*)tc::gemm_kernel<__nv_bfloat16> : (const void*)tc::gemm_kernel<__half>;
-  if (!attr_set[ti]) {
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES) != cudaSuccess)
-      return MUON_ERR_CUDA;
-    attr_set[ti] = true;
-  }
   Counters& cn = counters();
   cn.launches += 1;
   cn.gemm_launches += 1;
@@ -546,6 +539,14 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
     cn.flops_dense += 2.0 * mnk;
     cn.flops_sym += g.sym ? mnk : 2.0 * mnk;
     cn.flops_exec += 2.0 * tc::BM * tc::BN * (double)g.K * g.tiles_per_batch * g.batch;
+  }
+  static bool attr_set[2] = {false, false};
+  const int ti = t == Op::BF16 ? 0 : 1;
+  const void* fn = t == Op::BF16 ? (const void*)tc::gemm_kernel<__nv_bfloat16> : (const void*)tc::gemm_kernel<__half>;
+  if (!attr_set[ti]) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES) != cudaSuccess)
+      return MUON_ERR_CUDA;
+    attr_set[ti] = true;
   }
   const int grid = total < num_sms() ? total : num_sms();
   if (t == Op::BF16)
