@@ -46,6 +46,8 @@ WORKLOADS = {
                              compute="f16", gram=True, normuon=True, dion3=(1, 4)),
     "llama7b": dict(desc="Llama-7B layer set: 32 x (4 x 4096x4096, 4096x14336, 14336x4096), bf16 NS T=5",
                     compute="bf16", gram=False, normuon=False, dion3=None),
+    "llama_mlp_4096x14336": dict(desc="one Llama-7B MLP matrix 4096x14336, bf16 NS T=5 (profiling case)",
+                                 compute="bf16", gram=False, normuon=False, dion3=None),
     "llama7b_normuon": dict(desc="Llama-7B layer set, bf16 NS T=5, NorMuon on",
                             compute="bf16", gram=False, normuon=True, dion3=None),
     "spectrum4096x16384": dict(desc="one 4096x16384 bf16 matrix, singular values log-uniform in [1e-4, 1]: "
@@ -74,6 +76,8 @@ def specs_for(name: str):
         return inputs.gpt124m_layer_set()
     if name == "dion3_8192x28672":
         return [inputs.MatrixSpec(8192, 28672, 4000, "x")]
+    if name == "llama_mlp_4096x14336":
+        return [inputs.llama7b_layer_set()[4]]
     if name.startswith("llama7b"):
         return inputs.llama7b_layer_set()
     raise ValueError(name)
@@ -346,6 +350,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks,
         "device_status": mu.status_str(status),
         "cuda_graph": bool(args.graph),
+        "gemm": "cta_pair" if args.cta_pair else "single_cta",
     }
     return out
 
@@ -522,6 +527,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end arm")
     ap.add_argument("--graph", type=int, default=1, help="1: replay the step as one captured CUDA graph")
+    ap.add_argument("--cta-pair", type=int, default=1, help="1: CTA-pair tensor-core GEMM, 0: single-CTA")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -541,6 +547,8 @@ def main():
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    from newton_schulz_10_b200 import muon as mu
+    mu.set_gemm_cta_pair(bool(args.cta_pair))
     if args.workload == "spectrum4096x16384":
         out = run_spectrum(args, rank, world, local_rank)
     else:

@@ -123,6 +123,13 @@ typedef struct {
  * applies to launches queued after the call. */
 void muon_set_wait_timeout_ns(uint64_t ns);
 
+/* Tensor-core GEMM form used by the Newton-Schulz chain: 1 (default) runs
+ * each 256x256 tile on a pair of CTAs (tcgen05 cta_group::2, a cluster of two
+ * SMs, each loading half of the operands); 0 runs 128x256 tiles on single
+ * CTAs. Both give the same results up to fp32 summation order. Process-wide;
+ * applies to launches queued after the call. */
+void muon_set_gemm_cta_pair(int32_t enable);
+
 /* Human-readable name of a status value (static string, never NULL). */
 const char* muon_status_str(muon_status s);
 

@@ -459,6 +459,8 @@ extern "C" {
 
 void muon_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns ? ns : kDefaultTimeoutNs); }
 
+void muon_set_gemm_cta_pair(int32_t enable) { set_gemm_pair_mode(enable ? 2 : 1); }
+
 const char* muon_status_str(muon_status s) {
   switch (s) {
     case MUON_OK: return "MUON_OK";

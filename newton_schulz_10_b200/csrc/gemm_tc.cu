@@ -1,10 +1,19 @@
 // Tensor-core GEMM for the Newton-Schulz chain on sm_100a.
 //
-// Persistent, warp-specialised kernel: one CTA per SM, 384 threads.
-//   warp 0      TMA producer (one elected thread): A and B tiles into a
-//               4-stage shared-memory ring, 128-byte swizzle, no multicast
-//   warp 1      MMA issuer (one thread): tcgen05.mma kind::f16, 128x256x16
-//               per instruction, fp32 accumulator in TMEM
+// Persistent, warp-specialised kernel, one CTA per SM, 384 threads, in two
+// forms sharing everything but the mainloop's data movement:
+//   PAIR = 1  one CTA computes a 128x256 tile: tcgen05.mma cta_group::1,
+//             M = 128, N = 256; 4-stage ring of 48 KB (A 128x64, B 256x64).
+//   PAIR = 2  a cluster of two CTAs computes a 256x256 tile: the leader issues
+//             tcgen05.mma cta_group::2, M = 256, N = 256, reading A's 128 rows
+//             and B's 128 rows from each CTA's own shared memory; each CTA
+//             TMA-loads only its halves (32 KB per k-block instead of 48 KB
+//             of operand traffic per SM) into a 6-stage ring, and the copy
+//             completions are counted on the leader's barrier. MMA
+//             completions are signalled to both CTAs' barriers.
+// Roles:
+//   warp 0      TMA producer (one thread), 128-byte swizzle
+//   warp 1      MMA issuer (one thread of the leader), fp32 accumulators in TMEM
 //   warp 2      allocates / frees the 512 TMEM columns (two 128x256 fp32
 //               accumulators: the epilogue of tile i overlaps the mainloop of
 //               tile i+1)
@@ -20,14 +29,14 @@
 //
 // Symmetric outputs ("2. Symmetric GEMM Kernels" of the Dion3 page: a
 // triangular scheduler over lower tiles and a transposed-tile epilogue) are
-// scheduled over the 128x256 tiles that touch the lower triangle only.
+// scheduled over the tiles that touch the lower triangle only.
 //
 // Every wait is bounded (mbar_wait_bounded): on expiry the kernel records
 // MUON_ERR_TIMEOUT, every role stops, in-flight copies and MMAs are drained
 // with bounded waits and TMEM is freed before the CTA exits.
 #include <cstring>
-#include <type_traits>
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -36,24 +45,30 @@ namespace muon {
 
 namespace tc {
 
-constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int BM = 128, BN = 256, BK = 64;  // BM: rows per CTA
 constexpr int UMMA_K = 16;
-constexpr int A_STAGE = BM * BK * 2;  // 16 KB
-constexpr int B_STAGE = BN * BK * 2;  // 32 KB
 constexpr int EPI_WARP0 = 4;
 constexpr int EPI_WARPS = 8;                       // two per TMEM lane quarter
 constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
 constexpr int EPI_CHUNKS = BN / 32 / 2;            // 32-column chunks per epilogue warp
 constexpr int TMEM_COLS = 512;
-constexpr int EPI_BLOCK = 32 * 32 * 2;   // one staged 32x32 block of bf16/fp16, 64-byte rows
+constexpr int EPI_BLOCK = 32 * 32 * 2;             // one staged 32x32 block of bf16/fp16, 64-byte rows
+constexpr int EPI_BUF = 2 * EPI_BLOCK;             // per epilogue warp: direct block + mirrored block
 // Drains (in-flight copies and MMAs before exit) use their own bound, so that
 // a tiny configurable wait budget never lets a CTA exit with work in flight.
 constexpr uint64_t DRAIN_NS = 1000000000ull;
-constexpr int STAGES = 4;
-constexpr int EPI_BUF = 2 * EPI_BLOCK;  // per epilogue warp: direct block + mirrored block
-constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * (A_STAGE + B_STAGE) + EPI_WARPS * EPI_BUF +
-                           (2 * STAGES + 5) * 8 + 16;
-static_assert(SMEM_BYTES <= 232448, "exceeds the opt-in shared memory of one sm_100 CTA");
+
+template <int PAIR>
+struct Cfg {
+  static constexpr int STAGES = PAIR == 2 ? 6 : 4;
+  static constexpr int A_STAGE = BM * BK * 2;                  // this CTA's 128 rows of A
+  static constexpr int B_STAGE = (BN / PAIR) * BK * 2;         // this CTA's share of B's 256 rows
+  static constexpr int TX_BYTES = PAIR * (A_STAGE + B_STAGE);  // per stage, both CTAs
+  static constexpr int TILE_M = BM * PAIR;                     // rows of a (pair) tile
+  static constexpr int SMEM = 1024 /*align slack*/ + STAGES * (A_STAGE + B_STAGE) + EPI_WARPS * EPI_BUF +
+                              (2 * STAGES + 5) * 8 + 16;
+  static_assert(SMEM <= 232448, "exceeds the opt-in shared memory of one sm_100 CTA");
+};
 
 struct Group {
   CUtensorMap tmA;
@@ -79,14 +94,16 @@ struct Params {
 };
 
 struct Tile {
-  int g, b, m0, n0;
+  int g, b, m0, n0;  // m0: first row of the (pair) tile
 };
 
-__host__ __device__ inline int sym_row_tiles(int i, int tiles_n) {
-  int c = (i * BM + BM - 1) / BN + 1;
+// Tiles of row block i (tile_m rows) that touch the lower triangle.
+__host__ __device__ inline int sym_row_tiles(int i, int tiles_n, int tile_m) {
+  int c = (i * tile_m + tile_m - 1) / BN + 1;
   return c < tiles_n ? c : tiles_n;
 }
 
+template <int PAIR>
 __device__ inline Tile decode(const Params& p, int tile) {
   int gi = 0;
   while (gi + 1 < p.ngroups && tile >= p.g[gi + 1].tile_begin) ++gi;
@@ -101,7 +118,7 @@ __device__ inline Tile decode(const Params& p, int tile) {
   } else {
     int i = 0;
     for (;;) {
-      int cnt = sym_row_tiles(i, g.tiles_n);
+      int cnt = sym_row_tiles(i, g.tiles_n, Cfg<PAIR>::TILE_M);
       if (t < cnt) break;
       t -= cnt;
       ++i;
@@ -109,7 +126,7 @@ __device__ inline Tile decode(const Params& p, int tile) {
     tm = i;
     tn = t;
   }
-  return Tile{gi, b, tm * BM, tn * BN};
+  return Tile{gi, b, tm * Cfg<PAIR>::TILE_M, tn * BN};
 }
 
 __device__ __forceinline__ float powi(float s, int p) {
@@ -134,23 +151,40 @@ __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-template <typename T>
+// Spin (bounded) until the phase with this parity completed; for drains.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* status) {
+  const uint32_t addr = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(addr, parity)) {
+    if (globaltimer_ns() - t0 > DRAIN_NS) {
+      report(status, MUON_ERR_TIMEOUT);
+      break;
+    }
+  }
+}
+
+template <typename T, int PAIR>
 __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant__ Params p) {
+  using Cf = Cfg<PAIR>;
+  constexpr int STAGES = Cf::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_STAGE;
-  uint8_t* sEpi = sB + STAGES * B_STAGE;
+  uint8_t* sB = smem + STAGES * Cf::A_STAGE;
+  uint8_t* sEpi = sB + STAGES * Cf::B_STAGE;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + EPI_WARPS * EPI_BUF);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + STAGES;
+  uint64_t* full = bars;             // copies landed (the leader's counts both CTAs)
+  uint64_t* empty = bars + STAGES;   // MMAs finished reading the stage
   uint64_t* tfull = bars + 2 * STAGES;
-  uint64_t* tempty = tfull + 2;
+  uint64_t* tempty = tfull + 2;      // the leader's counts both CTAs' epilogues
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR == 2 ? cluster_rank() : 0;  // 0 = leader
+  const int unit = PAIR == 2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int units = PAIR == 2 ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -159,60 +193,73 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], EPI_WARPS * 32);
+      mbar_init(&tempty[b], EPI_WARPS * PAIR);  // one arrival per epilogue warp of the pair
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 2) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    if (PAIR == 2) {
+      tmem_alloc_pair(tmem_slot, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < p.ngroups; ++i) {
       prefetch_tmap(&p.g[i].tmA);
       prefetch_tmap(&p.g[i].tmB);
+      prefetch_tmap(&p.g[i].tmD);
     }
   }
   tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  if (PAIR == 2) cluster_sync(); else __syncthreads();  // barriers initialised in both CTAs
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint64_t budget = p.timeout_ns;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------------------
-    // TMA producer
+    // TMA producer (each CTA loads its own halves)
     // ------------------------------------------------------------------
     int stage = 0;
     uint32_t phase = 0;
     int issued = 0;
-    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
-      const Tile t = decode(p, tile);
+    for (int tile = unit; tile < p.total_tiles; tile += units) {
+      const Tile t = decode<PAIR>(p, tile);
       const Group& g = p.g[t.g];
       const int nkb = (g.K + BK - 1) / BK;
+      const int am0 = t.m0 + (int)rank * BM;            // this CTA's rows of A
+      const int bn0 = t.n0 + (int)rank * (BN / PAIR);   // this CTA's rows of B
       bool ok = true;
       for (int kb = 0; kb < nkb; ++kb) {
         if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, budget, p.status)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&full[stage], A_STAGE + B_STAGE);
-        uint8_t* a = sA + stage * A_STAGE;
-        uint8_t* b = sB + stage * B_STAGE;
+        if (rank == 0) mbar_arrive_expect_tx(&full[stage], Cf::TX_BYTES);
+        uint8_t* a = sA + stage * Cf::A_STAGE;
+        uint8_t* b = sB + stage * Cf::B_STAGE;
         const int k0 = kb * BK;
+        auto load = [&](void* dst, const CUtensorMap* m, int c0, int c1) {
+          if (PAIR == 2) tma_load_3d_pair(dst, m, c0, c1, t.b, &full[stage]);
+          else tma_load_3d(dst, m, c0, c1, t.b, &full[stage]);
+        };
         if (!g.a_mn) {
-          tma_load_3d(a, &g.tmA, k0, t.m0, t.b, &full[stage]);
+          load(a, &g.tmA, k0, am0);
         } else {
-          tma_load_3d(a, &g.tmA, t.m0, k0, t.b, &full[stage]);
-          tma_load_3d(a + 8192, &g.tmA, t.m0 + 64, k0, t.b, &full[stage]);
+          load(a, &g.tmA, am0, k0);
+          load(a + 8192, &g.tmA, am0 + 64, k0);
         }
         if (!g.b_mn) {
-          tma_load_3d(b, &g.tmB, k0, t.n0, t.b, &full[stage]);
+          load(b, &g.tmB, k0, bn0);
         } else {
 #pragma unroll
-          for (int j = 0; j < BN / 64; ++j) tma_load_3d(b + j * 8192, &g.tmB, t.n0 + 64 * j, k0, t.b, &full[stage]);
+          for (int j = 0; j < BN / PAIR / 64; ++j) load(b + j * 8192, &g.tmB, bn0 + 64 * j, k0);
         }
         ++issued;
         if (++stage == STAGES) {
@@ -222,39 +269,39 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       }
       if (!ok) break;
     }
-    // Drain: wait (bounded) until every copy issued into the ring landed.
-    int n = issued < STAGES ? issued : STAGES;
-    for (int i = 0; i < n; ++i) {
-      if (--stage < 0) {
-        stage = STAGES - 1;
-        phase ^= 1;
-      }
-      // the copies of the most recent use of `stage` completed phase `phase`
-      const uint32_t addr = smem_u32(&full[stage]);
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(addr, phase)) {
-        if (globaltimer_ns() - t0 > DRAIN_NS) {
-          report(p.status, MUON_ERR_TIMEOUT);
-          break;
+    if (PAIR == 1) {
+      // Drain: wait (bounded) until every copy issued into the ring landed.
+      int n = issued < STAGES ? issued : STAGES;
+      for (int i = 0; i < n; ++i) {
+        if (--stage < 0) {
+          stage = STAGES - 1;
+          phase ^= 1;
         }
+        drain_wait(&full[stage], phase, p.status);  // the most recent use of `stage`
+      }
+    } else if (*abort_flag) {
+      // The pair's copies complete on the leader's barriers, which this CTA
+      // cannot poll; on an early exit give in-flight copies time to land.
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 200000ull) {
       }
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1 && lane == 0 && rank == 0) {
     // ------------------------------------------------------------------
-    // MMA issuer
+    // MMA issuer (the leader issues for the pair)
     // ------------------------------------------------------------------
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
-    constexpr int fmt = sizeof(T) == 2 && std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
+    constexpr int fmt = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < p.total_tiles && ok; tile += gridDim.x) {
-      const Tile t = decode(p, tile);
+    for (int tile = unit; tile < p.total_tiles && ok; tile += units) {
+      const Tile t = decode<PAIR>(p, tile);
       const Group& g = p.g[t.g];
       const int nkb = (g.K + BK - 1) / BK;
-      const uint32_t idesc = idesc_f16(fmt, g.a_mn, g.b_mn, BM, BN);
+      const uint32_t idesc = idesc_f16(fmt, g.a_mn, g.b_mn, BM * PAIR, BN);
       // K-major: 8-row groups 1024 B apart, one K step = 32 B inside the
       // swizzle atom. MN-major: 64-element MN atoms 8 KB apart (LBO), 8-row
       // K groups 1024 B apart (SBO), one K step of 16 rows = 2048 B.
@@ -269,36 +316,37 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
           break;
         }
         tc_fence_after();
-        const uint32_t a_addr = a_base + stage * A_STAGE, b_addr = b_base + stage * B_STAGE;
+        const uint32_t a_addr = a_base + stage * Cf::A_STAGE, b_addr = b_base + stage * Cf::B_STAGE;
 #pragma unroll
         for (int k = 0; k < BK / UMMA_K; ++k) {
           const uint64_t ad = smem_desc_sw128(a_addr + k * a_kstep, a_lbo, 1024);
           const uint64_t bd = smem_desc_sw128(b_addr + k * b_kstep, b_lbo, 1024);
-          umma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          if (PAIR == 2) umma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          else umma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0);
         }
-        umma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
+        // frees the stage (in both CTAs) once these MMAs have read it
+        if (PAIR == 2) umma_commit_pair(&empty[stage], 0x3); else umma_commit(&empty[stage]);
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1;
         }
       }
       if (!ok) break;
-      umma_commit(&tfull[acc]);  // accumulator ready for the epilogue
+      // accumulator ready for the epilogue (of both CTAs)
+      if (PAIR == 2) umma_commit_pair(&tfull[acc], 0x3); else umma_commit(&tfull[acc]);
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
       }
     }
-    // Drain: every MMA issued by this thread completes before TMEM is freed.
-    umma_commit(drain);
-    const uint32_t addr = smem_u32(drain);
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(addr, 0)) {
-      if (globaltimer_ns() - t0 > DRAIN_NS) {
-        report(p.status, MUON_ERR_TIMEOUT);
-        break;
-      }
-    }
+    // Drain: every MMA issued completes (and every earlier completion signal
+    // has arrived) before TMEM is freed.
+    if (PAIR == 2) umma_commit_pair(drain, 0x3); else umma_commit(drain);
+    drain_wait(drain, 0, p.status);
+  } else if (PAIR == 2 && warp == 1 && lane == 0) {
+    // the follower learns from the leader's drain signal that no MMA still
+    // reads its shared memory or writes its TMEM
+    drain_wait(drain, 0, p.status);
   } else if (warp >= EPI_WARP0) {
     // ------------------------------------------------------------------
     // Epilogue
@@ -310,8 +358,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     uint8_t* const sm = sd + EPI_BLOCK;       // staged mirrored block
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
-      const Tile t = decode(p, tile);
+    for (int tile = unit; tile < p.total_tiles; tile += units) {
+      const Tile t = decode<PAIR>(p, tile);
       const Group& g = p.g[t.g];
       // every lane waits; the verdict is made warp-uniform so the warp-wide
       // tcgen05.ld below never runs with part of the warp gone
@@ -321,7 +369,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       const float s = g.scale ? g.scale[t.b] : 1.f;
       const float alpha = g.alpha * powi(s, g.alpha_pow);
       const float beta = g.beta * powi(s, g.beta_pow);
-      const int r0 = t.m0 + q * 32;
+      const int r0 = t.m0 + (int)rank * BM + q * 32;
       const int row = r0 + lane;
       const int cbase = t.n0 + half * (BN / 2);
       // The C rows this thread needs, loaded for all its chunks before the
@@ -402,8 +450,13 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
           bulk_commit();
         }
       }
+      // this warp's TMEM reads are done: release the accumulator (to the leader)
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      __syncwarp();
+      if (lane == 0) {
+        if (PAIR == 2) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+        else mbar_arrive(&tempty[acc]);
+      }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
@@ -413,9 +466,13 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
   }
 
   tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  if (PAIR == 2) cluster_sync(); else __syncthreads();  // no CTA leaves while its pair still signals it
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (warp == 2) {
+    if (PAIR == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
+  }
 }
 
 }  // namespace tc
@@ -461,6 +518,54 @@ bool make_map(CUtensorMap* m, Op t, const void* base, int64_t inner, int64_t out
   return r == CUDA_SUCCESS;
 }
 
+template <typename T, int PAIR>
+muon_status launch(const tc::Params& p, int total_tiles, cudaStream_t s) {
+  static bool attr_set = false;
+  static int max_units = 0;  // co-resident CTAs (PAIR = 1) or clusters (PAIR = 2)
+  const void* fn = (const void*)tc::gemm_kernel<T, PAIR>;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Cfg<PAIR>::SMEM) != cudaSuccess)
+      return MUON_ERR_CUDA;
+    max_units = num_sms() / PAIR;
+    if (PAIR == 2) {
+      // not every SM may have a free partner in its GPC: launch only as many
+      // persistent pairs as can run at once
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3(2 * max_units);
+      q.blockDim = dim3(tc::THREADS);
+      q.dynamicSmemBytes = tc::Cfg<PAIR>::SMEM;
+      cudaLaunchAttribute a[1];
+      a[0].id = cudaLaunchAttributeClusterDimension;
+      a[0].val.clusterDim.x = 2;
+      a[0].val.clusterDim.y = 1;
+      a[0].val.clusterDim.z = 1;
+      q.attrs = a;
+      q.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, fn, &q) == cudaSuccess && clusters > 0 && clusters < max_units)
+        max_units = clusters;
+      cudaGetLastError();
+    }
+    attr_set = true;
+  }
+  const int units = total_tiles < max_units ? total_tiles : max_units;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(units * PAIR);
+  cfg.blockDim = dim3(tc::THREADS);
+  cfg.dynamicSmemBytes = tc::Cfg<PAIR>::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = PAIR;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc::gemm_kernel<T, PAIR>, p) == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
+}
+
+int g_pair_mode = 2;  // 2: CTA-pair kernel, 1: single-CTA kernel
+
 }  // namespace
 
 int num_sms() {
@@ -473,8 +578,12 @@ int num_sms() {
   return n;
 }
 
+void set_gemm_pair_mode(int pair) { g_pair_mode = pair == 1 ? 1 : 2; }
+
 muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t timeout_ns, cudaStream_t s) {
   if (ngroups < 1 || ngroups > kMaxGemmGroups || (t != Op::BF16 && t != Op::F16)) return MUON_ERR_INVALID_ARG;
+  const int pair = g_pair_mode;
+  const int tile_m = tc::BM * pair;
   tc::Params p;
   memset(&p, 0, sizeof(p));
   int total = 0;
@@ -485,11 +594,12 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
     if (d.ldd % 64 || (d.beta != 0.f && d.ldc % 64)) return MUON_ERR_INVALID_ARG;
     if (d.sym && d.M != d.N) return MUON_ERR_INVALID_ARG;
     tc::Group& g = p.g[ng];
-    // A operand source: K-major [M][K], MN-major [K][M]
+    // A operand source: K-major [M][K], MN-major [K][M]; 128 rows per CTA.
+    // B operand source: K-major [N][K], MN-major [K][N]; 256 / pair rows per CTA.
     bool ok = d.a_mn ? make_map(&g.tmA, t, d.A, d.M, d.K, d.batch, d.lda, d.strideA, 64)
                      : make_map(&g.tmA, t, d.A, d.K, d.M, d.batch, d.lda, d.strideA, tc::BM);
     ok = ok && (d.b_mn ? make_map(&g.tmB, t, d.B, d.N, d.K, d.batch, d.ldb, d.strideB, 64)
-                       : make_map(&g.tmB, t, d.B, d.K, d.N, d.batch, d.ldb, d.strideB, tc::BN));
+                       : make_map(&g.tmB, t, d.B, d.K, d.N, d.batch, d.ldb, d.strideB, tc::BN / pair));
     ok = ok && make_map(&g.tmD, t, d.D, d.N, d.M, d.batch, d.ldd, d.strideD, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
     if (!ok) return MUON_ERR_CUDA;
     g.D = d.D;
@@ -511,11 +621,11 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
     g.alpha = d.alpha;
     g.beta = d.beta;
     g.gamma = d.gamma;
-    g.tiles_m = (d.M + tc::BM - 1) / tc::BM;
+    g.tiles_m = (d.M + tile_m - 1) / tile_m;
     g.tiles_n = (d.N + tc::BN - 1) / tc::BN;
     if (d.sym) {
       int c = 0;
-      for (int i2 = 0; i2 < g.tiles_m; ++i2) c += tc::sym_row_tiles(i2, g.tiles_n);
+      for (int i2 = 0; i2 < g.tiles_m; ++i2) c += tc::sym_row_tiles(i2, g.tiles_n, tile_m);
       g.tiles_per_batch = c;
     } else {
       g.tiles_per_batch = g.tiles_m * g.tiles_n;
@@ -538,22 +648,11 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
     const double mnk = (double)g.M * g.N * g.K * g.batch;
     cn.flops_dense += 2.0 * mnk;
     cn.flops_sym += g.sym ? mnk : 2.0 * mnk;
-    cn.flops_exec += 2.0 * tc::BM * tc::BN * (double)g.K * g.tiles_per_batch * g.batch;
+    cn.flops_exec += 2.0 * tile_m * tc::BN * (double)g.K * g.tiles_per_batch * g.batch;
   }
-  static bool attr_set[2] = {false, false};
-  const int ti = t == Op::BF16 ? 0 : 1;
-  const void* fn = t == Op::BF16 ? (const void*)tc::gemm_kernel<__nv_bfloat16> : (const void*)tc::gemm_kernel<__half>;
-  if (!attr_set[ti]) {
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES) != cudaSuccess)
-      return MUON_ERR_CUDA;
-    attr_set[ti] = true;
-  }
-  const int grid = total < num_sms() ? total : num_sms();
-  if (t == Op::BF16)
-    tc::gemm_kernel<__nv_bfloat16><<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(p);
-  else
-    tc::gemm_kernel<__half><<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(p);
-  return cudaGetLastError() == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
+  if (pair == 2)
+    return t == Op::BF16 ? launch<__nv_bfloat16, 2>(p, total, s) : launch<__half, 2>(p, total, s);
+  return t == Op::BF16 ? launch<__nv_bfloat16, 1>(p, total, s) : launch<__half, 1>(p, total, s);
 }
 
 }  // namespace muon

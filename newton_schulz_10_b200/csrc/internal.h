@@ -54,6 +54,9 @@ muon_status simt_gemm(const GemmDesc& g, cudaStream_t s);
 
 int num_sms();
 
+// 2: tensor-core GEMMs use the CTA-pair kernel (default); 1: single-CTA kernel.
+void set_gemm_pair_mode(int pair);
+
 // Per-thread accounting of queued work (launch counts, NS FLOPs).
 struct Counters {
   int64_t launches = 0;

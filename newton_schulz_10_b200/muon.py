@@ -24,7 +24,7 @@ F32, BF16, F16 = 0, 1, 2
 # muon_norm
 NORM_L1, NORM_L2 = 0, 1
 
-EXPORTS = ("muon_set_wait_timeout_ns", "muon_status_str", "muon_rows_for_fraction", "muon_ns_params_default",
+EXPORTS = ("muon_set_wait_timeout_ns", "muon_set_gemm_cta_pair", "muon_status_str", "muon_rows_for_fraction", "muon_ns_params_default",
            "muon_ns_workspace_size", "ns_polar", "gram_ns_polar", "normuon_scale", "muon_select_workspace_size",
            "select_rows", "muon_workspace_size", "muon_step", "muon_step_profiled", "muon_kernel_launch_count",
            "select_rows_noalloc")
@@ -76,6 +76,8 @@ def lib() -> C.CDLL:
         vp, i32, i64, sz, f32 = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t, C.c_float
         L.muon_set_wait_timeout_ns.argtypes = [C.c_uint64]
         L.muon_set_wait_timeout_ns.restype = None
+        L.muon_set_gemm_cta_pair.argtypes = [i32]
+        L.muon_set_gemm_cta_pair.restype = None
         L.muon_status_str.argtypes = [i32]
         L.muon_status_str.restype = C.c_char_p
         L.muon_rows_for_fraction.argtypes = [i64, i32, i32]
@@ -186,6 +188,11 @@ def workspace(nbytes: int, device=None):
 def kernel_launch_count() -> int:
     """Kernels this library queued from the calling thread so far."""
     return lib().muon_kernel_launch_count()
+
+
+def set_gemm_cta_pair(enable: bool) -> None:
+    """True (default): CTA-pair tensor-core GEMM; False: single-CTA kernel."""
+    lib().muon_set_gemm_cta_pair(int(bool(enable)))
 
 
 def set_wait_timeout_ns(ns: int) -> None:
