@@ -185,6 +185,19 @@ class ClockSampler:
                 "in_region": any(t0 <= r[0] <= t1 for r in rows)}
 
 
+def max_over_ranks(value: float, world: int) -> float:
+    """Max of a per-rank number over all ranks (the reported time of a
+    multi-GPU run is the slowest rank's)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -228,11 +241,7 @@ def end_to_end(args, state, run, stream, elems, big, world):
             hw.copy_(W, non_blocking=True)
     f1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1) / e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / e2e_steps, world)
     return {"value": round(e2e_ms, 3), "unit": "ms/step", "h2d_bytes_per_step": 4 * elems,
             "d2h_bytes_per_step": 4 * elems, "what": "G pinned-host->device, step, W device->pinned-host",
             "steps": e2e_steps}
@@ -298,11 +307,7 @@ def run_ours(args, rank, world, local_rank):
         launches = args.steps * step.profiled(stream).kernel_launches
     if world > 1:
         dist.barrier()
-    ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        tt = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
     clocks = clk.summary(t0, t1)
 
     # --- per-phase profile (separate, untimed run) --------------------------
@@ -391,11 +396,7 @@ def run_spectrum(args, rank, world, local_rank):
             e1.record(stream)
             torch.cuda.synchronize()
             t1 = time.time()
-        ms = e0.elapsed_time(e1) / args.steps
-        if world > 1:
-            tt = torch.tensor([ms], device="cuda")
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ms = float(tt.item())
+        ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
         if name == "gram_f16":
             clocks = clk.summary(t0, t1)
             launches = mu.kernel_launch_count() - n0
