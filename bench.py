@@ -529,6 +529,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end arm")
     ap.add_argument("--graph", type=int, default=1, help="1: replay the step as one captured CUDA graph")
     ap.add_argument("--cta-pair", type=int, default=1, help="1: CTA-pair tensor-core GEMM, 0: single-CTA")
+    ap.add_argument("--wait-timeout-ms", type=float, default=0.0, help="bound of device-side waits (0: default)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -550,6 +551,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     from newton_schulz_10_b200 import muon as mu
     mu.set_gemm_cta_pair(bool(args.cta_pair))
+    if args.wait_timeout_ms > 0:
+        mu.set_wait_timeout_ns(int(args.wait_timeout_ms * 1e6))
     if args.workload == "spectrum4096x16384":
         out = run_spectrum(args, rank, world, local_rank)
     else:

@@ -12,7 +12,7 @@
 //             completions are counted on the leader's barrier. MMA
 //             completions are signalled to both CTAs' barriers.
 // Roles:
-//   warp 0      TMA producer (one thread), 128-byte swizzle
+//   warps 0, 3  TMA producers (one thread each: A boxes, B boxes), 128-byte swizzle
 //   warp 1      MMA issuer (one thread of the leader), fp32 accumulators in TMEM
 //   warp 2      allocates / frees the 512 TMEM columns (two 128x256 fp32
 //               accumulators: the epilogue of tile i overlaps the mainloop of
@@ -222,10 +222,16 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
   const uint32_t tmem_base = *tmem_slot;
   const uint64_t budget = p.timeout_ns;
 
-  if (warp == 0 && lane == 0) {
+  if ((warp == 0 || warp == 3) && lane == 0) {
     // ------------------------------------------------------------------
-    // TMA producer (each CTA loads its own halves)
+    // TMA producers (each CTA loads its own halves). Issuing a tensor copy
+    // costs the issuing thread hundreds of cycles, so two threads in
+    // different warps issue in parallel: warp 0 the A boxes (and the
+    // leader's byte count), warp 3 the B boxes. Each of them has a box in
+    // every k-block, so no stage phase can complete without both, and
+    // neither can fall two phases behind the parity it waits on.
     // ------------------------------------------------------------------
+    const bool issues_a = warp == 0;
     int stage = 0;
     uint32_t phase = 0;
     int issued = 0;
@@ -241,7 +247,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
           ok = false;
           break;
         }
-        if (rank == 0) mbar_arrive_expect_tx(&full[stage], Cf::TX_BYTES);
+        if (issues_a && rank == 0) mbar_arrive_expect_tx(&full[stage], Cf::TX_BYTES);
         uint8_t* a = sA + stage * Cf::A_STAGE;
         uint8_t* b = sB + stage * Cf::B_STAGE;
         const int k0 = kb * BK;
@@ -249,17 +255,20 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
           if (PAIR == 2) tma_load_3d_pair(dst, m, c0, c1, t.b, &full[stage]);
           else tma_load_3d(dst, m, c0, c1, t.b, &full[stage]);
         };
-        if (!g.a_mn) {
-          load(a, &g.tmA, k0, am0);
+        if (issues_a) {
+          if (!g.a_mn) {
+            load(a, &g.tmA, k0, am0);
+          } else {
+            load(a, &g.tmA, am0, k0);
+            load(a + 8192, &g.tmA, am0 + 64, k0);
+          }
         } else {
-          load(a, &g.tmA, am0, k0);
-          load(a + 8192, &g.tmA, am0 + 64, k0);
-        }
-        if (!g.b_mn) {
-          load(b, &g.tmB, k0, bn0);
-        } else {
+          if (!g.b_mn) {
+            load(b, &g.tmB, k0, bn0);
+          } else {
 #pragma unroll
-          for (int j = 0; j < BN / PAIR / 64; ++j) load(b + j * 8192, &g.tmB, bn0 + 64 * j, k0);
+            for (int j = 0; j < BN / PAIR / 64; ++j) load(b + j * 8192, &g.tmB, bn0 + 64 * j, k0);
+          }
         }
         ++issued;
         if (++stage == STAGES) {

@@ -350,3 +350,21 @@ def test_step_cuda_graph_matches_eager():
     for a, b in zip(d1, d2):
         for x, y in zip(a, b):
             assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("pair", [True, False])
+def test_step_many_tiles_mixed_layouts(pair):
+    """More tiles than persistent CTAs (or CTA pairs), with wide, square and
+    tall groups (K-major and MN-major operands) sharing every launch: each
+    CTA walks many tiles of different layouts through one shared-memory ring,
+    the case where producer/consumer phase tracking must hold up."""
+    shapes = [(512, 512)] * 40 + [(512, 1536)] * 8 + [(1536, 512)] * 8
+    state = make_state(shapes, 8000, m_std=1e-3)
+    mu.set_gemm_cta_pair(pair)
+    try:
+        got, st = run_step(state, mu.step_params())
+    finally:
+        mu.set_gemm_cta_pair(True)
+    assert st == mu.OK, mu.status_str(st)
+    idx = [0, 39, 40, 47, 48, 55]
+    check_step([state[i] for i in idx], [got[i] for i in idx], O.StepParams(), TOL16)
