@@ -144,7 +144,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
             time.sleep(0.3)
@@ -196,6 +196,28 @@ def max_over_ranks(value: float, world: int) -> float:
     t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def gemm_traffic(workload: str):
+    """Mean DRAM bytes per GEMM launch from the committed ncu summary of this
+    workload, if the kernel sources are unchanged since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"gemm_kernel_{workload}.md")
+    if not os.path.exists(path):
+        return None, None
+    want = traffic = None
+    for line in open(path):
+        if line.startswith("source-sha256:"):
+            want = line.split(":", 1)[1].strip()
+        elif line.startswith("dram-bytes-per-launch:"):
+            traffic = float(line.split(":", 1)[1])
+    h = hashlib.sha256()
+    for f in ("gemm_tc.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "newton_schulz_10_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if want is None or traffic is None or h.hexdigest()[:16] != want:
+        return None, None
+    return traffic, os.path.relpath(path, ROOT)
 
 
 def measured_peaks():
@@ -325,9 +347,13 @@ def run_ours(args, rank, world, local_rank):
         roof = None
     else:
         achieved = prof.ns_flops / (prof.ms_ns * 1e-3) / 1e12
+        traffic, traffic_src = gemm_traffic(args.workload)
         roof = {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 NS chain)", "achieved": round(achieved, 1),
                 "peak": tensor_peak, "unit": "TFLOP/s", "frac": round(achieved / tensor_peak, 4),
-                "traffic": None, "peak_source": f"{peak_kind} {'sustained' if long_step else 'burst'} bf16",
+                "traffic": traffic, "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
+                "traffic_source": traffic_src,
+                "flops_per_launch_algorithmic": prof.ns_flops / max(prof.gemm_launches, 1),
+                "peak_source": f"{peak_kind} {'sustained' if long_step else 'burst'} bf16",
                 "flops_per_step_algorithmic": prof.ns_flops, "flops_per_step_executed": prof.ns_flops_executed,
                 "gemm_launches_per_step": prof.gemm_launches,
                 "achieved_executed": round(prof.ns_flops_executed / (prof.ms_ns * 1e-3) / 1e12, 1)}
@@ -520,7 +546,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt124m")
