@@ -12,6 +12,7 @@ namespace muon {
 namespace {
 
 constexpr int BLOCK = 256;
+constexpr int UNROLL = 4;  // momentum pass: 16-byte vectors of M and G in flight per lane
 
 __device__ __forceinline__ int find_mat(const RowLaunch& L, int task) {
   int lo = 0, hi = L.count - 1;
@@ -93,19 +94,34 @@ __global__ void __launch_bounds__(BLOCK) momentum_rows(const __grid_constant__ R
     const float mu = L.mu;
     if ((m.cols & 3) == 0) {
       const int64_t n4 = m.cols >> 2;
-      for (int64_t c = l; c < n4; c += WG) {
-        float4 x = *reinterpret_cast<const float4*>(M + 4 * c);
-        const float4 g = __ldcs(reinterpret_cast<const float4*>(G + 4 * c));
-        if (MODE == MOM_MUON) {
-          x.x = fmaf(mu, x.x, g.x); x.y = fmaf(mu, x.y, g.y); x.z = fmaf(mu, x.z, g.z); x.w = fmaf(mu, x.w, g.w);
-        } else {
-          x.x += g.x; x.y += g.y; x.z += g.z; x.w += g.w;
+      // UNROLL vectors of M and of G in flight per lane before any is used
+      for (int64_t c0 = l; c0 < n4; c0 += UNROLL * WG) {
+        float4 x[UNROLL], g[UNROLL];
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+          const int64_t c = c0 + u * WG;
+          if (c < n4) {
+            x[u] = *reinterpret_cast<const float4*>(M + 4 * c);
+            g[u] = __ldcs(reinterpret_cast<const float4*>(G + 4 * c));
+          }
         }
-        *reinterpret_cast<float4*>(M + 4 * c) = x;
-        if (CAST) Dst<T>::store4(X + 4 * c, x);
-        const double a = x.x, b = x.y, cc = x.z, d = x.w;
-        ss += a * a + b * b + cc * cc + d * d;
-        sa += fabs(a) + fabs(b) + fabs(cc) + fabs(d);
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+          const int64_t c = c0 + u * WG;
+          if (c >= n4) break;
+          float4 y = x[u];
+          if (MODE == MOM_MUON) {
+            y.x = fmaf(mu, y.x, g[u].x); y.y = fmaf(mu, y.y, g[u].y);
+            y.z = fmaf(mu, y.z, g[u].z); y.w = fmaf(mu, y.w, g[u].w);
+          } else {
+            y.x += g[u].x; y.y += g[u].y; y.z += g[u].z; y.w += g[u].w;
+          }
+          *reinterpret_cast<float4*>(M + 4 * c) = y;
+          if (CAST) Dst<T>::store4(X + 4 * c, y);
+          const double a = y.x, b = y.y, cc = y.z, d = y.w;
+          ss += a * a + b * b + cc * cc + d * d;
+          sa += fabs(a) + fabs(b) + fabs(cc) + fabs(d);
+        }
       }
     } else {
       for (int64_t c = l; c < m.cols; c += WG) {
