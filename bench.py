@@ -53,6 +53,9 @@ WORKLOADS = {
     "spectrum4096x16384": dict(desc="one 4096x16384 bf16 matrix, singular values log-uniform in [1e-4, 1]: "
                                     "Gram NS (fp16, restart 3) vs standard NS (bf16 and fp16), T=5",
                                compute="f16", gram=True, normuon=False, dion3=None),
+    "moe_alpha8_2048x16384": dict(desc="one MoE-shaped 2048x16384 bf16 matrix (aspect ratio 8, Gaussian): "
+                                       "Gram NS (fp16, restart 3) vs standard NS (bf16 and fp16), T=5",
+                                  compute="f16", gram=True, normuon=False, dion3=None),
 }
 
 
@@ -70,6 +73,8 @@ def ns_flops(n, m, T, gram, restart_at=3):
 def specs_for(name: str):
     if name == "spectrum4096x16384":
         return [inputs.MatrixSpec(4096, 16384, 3000, "x")]
+    if name == "moe_alpha8_2048x16384":
+        return [inputs.MatrixSpec(2048, 16384, 6000, "x")]
     if name == "single256x1024":
         return [inputs.MatrixSpec(256, 1024, 1000, "x")]
     if name == "gpt124m":
@@ -229,44 +234,64 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def end_to_end(args, state, run, stream, elems, big, world):
-    """Same step with host buffers: each step copies that step's gradients
-    from pinned host memory to the device and the updated weights back."""
+def end_to_end(args, state, step, stream, elems, big, world):
+    """The step as a training loop drives it, through the public API with
+    host buffers: every step's gradients are copied from pinned host memory
+    to the device (on a copy stream, into one of two device buffers, so the
+    upload of step k+1 overlaps step k), the step runs, and its result, the
+    4-byte device status word, is read back to pinned host memory. W, M and v
+    stay resident, as optimizer state does in training."""
     import torch
     import torch.distributed as dist
 
-    # each step: H2D copy of that step's gradients from pinned memory, the
-    # step, D2H copy of the updated weights into pinned memory
+    from newton_schulz_10_b200 import muon as mu
+
     try:
         import psutil
         avail = psutil.virtual_memory().available
     except ImportError:
         avail = 1 << 62
-    if 2 * 4 * elems > 0.5 * avail:
-        return {"value": None, "unit": "ms/step", "h2d_bytes_per_step": 4 * elems, "d2h_bytes_per_step": 4 * elems,
-                "reason": f"pinned host buffers need {8 * elems / 1e9:.1f} GB, {avail / 1e9:.1f} GB available"}
+    if 4 * elems > 0.5 * avail:
+        return {"value": None, "unit": "ms/step", "h2d_bytes_per_step": 4 * elems, "d2h_bytes_per_step": 4,
+                "reason": f"pinned host gradients need {4 * elems / 1e9:.1f} GB, {avail / 1e9:.1f} GB available"}
     hostG = [torch.empty_like(G, device="cpu").pin_memory() for (_, _, G, _) in state]
-    hostW = [torch.empty_like(W, device="cpu").pin_memory() for (W, _, _, _) in state]
     for hg, (_, _, G, _) in zip(hostG, state):
         hg.copy_(G)
-    e2e_steps = max(1, min(args.steps, 20 if not big else 3))
+    # second device gradient buffer and a step bound to it (same workspace)
+    G2 = [torch.empty_like(G) for (_, _, G, _) in state]
+    steps = [step, mu.Step([(W, M, g2, v) for (W, M, _, v), g2 in zip(state, G2)], step.params, ws=step.ws)]
+    gsets = [[G for (_, _, G, _) in state], G2]
+    status_host = torch.zeros(1, dtype=torch.int32).pin_memory()
+    copy_stream = torch.cuda.Stream()
+    copied = [torch.cuda.Event(), torch.cuda.Event()]
+    done = [torch.cuda.Event(), torch.cuda.Event()]
+    e2e_steps = max(2, min(args.steps, 50 if not big else 4))
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(stream)
-    for _ in range(e2e_steps):
-        for hg, (_, _, G, _) in zip(hostG, state):
-            G.copy_(hg, non_blocking=True)
-        run(stream)
-        for hw, (W, _, _, _) in zip(hostW, state):
-            hw.copy_(W, non_blocking=True)
+    copy_stream.wait_event(f0)
+    for k in range(e2e_steps):
+        buf = k % 2
+        with torch.cuda.stream(copy_stream):
+            if k >= 2:
+                copy_stream.wait_event(done[buf])  # step k-2 has finished reading this buffer
+            for hg, g in zip(hostG, gsets[buf]):
+                g.copy_(hg, non_blocking=True)
+            copied[buf].record(copy_stream)
+        stream.wait_event(copied[buf])
+        steps[buf](stream)
+        done[buf].record(stream)
+        with torch.cuda.stream(stream):
+            status_host.copy_(steps[buf].ws[:4].view(torch.int32), non_blocking=True)
     f1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1) / e2e_steps, world)
-    return {"value": round(e2e_ms, 3), "unit": "ms/step", "h2d_bytes_per_step": 4 * elems,
-            "d2h_bytes_per_step": 4 * elems, "what": "G pinned-host->device, step, W device->pinned-host",
-            "steps": e2e_steps}
+    return {"value": round(e2e_ms, 3), "unit": "ms/step", "h2d_bytes_per_step": 4 * elems, "d2h_bytes_per_step": 4,
+            "what": "G pinned host -> device on a copy stream (double-buffered, overlapping the previous step), "
+                    "step, 4-byte status word -> pinned host",
+            "steps": e2e_steps, "status": mu.status_str(int(status_host.item()))}
 
 
 # ---------------------------------------------------------------------------
@@ -339,7 +364,7 @@ def run_ours(args, rank, world, local_rank):
     if args.no_e2e:
         e2e = None
     else:
-        e2e = end_to_end(args, state, run, stream, elems, big, world)
+        e2e = end_to_end(args, state, step, stream, elems, big, world)
     peaks, peak_kind = measured_peaks()
     long_step = ms > 100.0
     tensor_peak = peaks["bf16_tflops_sustained" if long_step else "bf16_tflops"]
@@ -387,17 +412,22 @@ def run_ours(args, rank, world, local_rank):
 
 
 def run_spectrum(args, rank, world, local_rank):
-    """Gram vs standard Newton-Schulz on the 4096 x 16384 spectrum matrix."""
+    """Gram vs standard Newton-Schulz on one matrix: the 4096 x 16384
+    spectrum matrix, or the 2048 x 16384 MoE-shaped Gaussian matrix."""
     import torch
     import torch.distributed as dist
 
     from newton_schulz_10_b200 import muon as mu
 
     torch.cuda.set_device(local_rank)
-    X, _ = inputs.spectrum_matrix(4096, 16384, -4.0, seed=3000)
+    if args.workload == "spectrum4096x16384":
+        n, m = 4096, 16384
+        X, _ = inputs.spectrum_matrix(n, m, -4.0, seed=3000)
+    else:
+        n, m = 2048, 16384
+        X = inputs.gaussian((n, m), 1.0, 6000, 0)
     Xd = torch.from_numpy(X.astype(np.float32)).cuda().to(torch.bfloat16)
     del X
-    n, m = 4096, 16384
     variants = [("gram_f16", mu.ns_params(gram=True, restart_at=3, compute=mu.F16), True),
                 ("standard_bf16", mu.ns_params(compute=mu.BF16), False),
                 ("standard_f16", mu.ns_params(compute=mu.F16), False)]
@@ -442,12 +472,13 @@ def run_spectrum(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": g["ms"], "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
         "config": {"workload": args.workload, "description": cfg["desc"], "step": "one gram_ns_polar call",
-                   "l2": "operands 128 MiB bf16 input + 256 MiB working set, larger than L2"},
+                   "l2": f"bf16 input {2 * n * m / 2**20:.0f} MiB plus working set, larger than L2"},
         "roofline": {"bound": "tensor", "kernel": "gemm_kernel (Gram NS chain)", "achieved": g["tflops_algorithmic"],
                      "peak": peak, "unit": "TFLOP/s", "frac": round(g["tflops_algorithmic"] / peak, 4),
                      "traffic": None, "peak_source": f"{kind} burst bf16 (fp16 has the same dense rate)"},
         "variants": res,
         "speedup_gram_vs_standard_bf16": round(res["standard_bf16"]["ms"] / g["ms"], 3),
+        "flop_ratio_standard_over_gram": round(ns_flops(n, m, 5, False) / ns_flops(n, m, 5, True), 3),
         "e2e": None, "gpu_launches": launches, "clocks": clocks,
     }
 
@@ -464,6 +495,14 @@ def oracle_sample(workload: str, budget_s: float):
 
     cfg = WORKLOADS[workload]
     specs = specs_for(workload)
+    if workload == "moe_alpha8_2048x16384":
+        X = inputs.gaussian((512, 4096), 1.0, 6000, 0).astype(np.float64)
+        t = time.perf_counter()
+        oracle.gram_newton_schulz(X, (COEFFS,) * 5, 1e-7, 3)
+        dt = time.perf_counter() - t
+        scale = ns_flops(2048, 16384, 5, True) / ns_flops(512, 4096, 5, True)
+        return 1e3 * dt * scale, (f"oracle gram_newton_schulz on a 512x4096 Gaussian matrix (aspect 8), "
+                                  f"{dt:.2f} s, scaled x{scale:.0f} by the Gram FLOP formula"), threads_used()
     if workload == "spectrum4096x16384":
         t = time.perf_counter()
         X, _ = inputs.spectrum_matrix(1024, 4096, -4.0, seed=3000)
@@ -579,7 +618,7 @@ def main():
     mu.set_gemm_cta_pair(bool(args.cta_pair))
     if args.wait_timeout_ms > 0:
         mu.set_wait_timeout_ns(int(args.wait_timeout_ms * 1e6))
-    if args.workload == "spectrum4096x16384":
+    if args.workload in ("spectrum4096x16384", "moe_alpha8_2048x16384"):
         out = run_spectrum(args, rank, world, local_rank)
     else:
         out = run_ours(args, rank, world, local_rank)
