@@ -66,6 +66,7 @@ float rho_for(Op t, int64_t n) { return t == Op::F16 ? (float)n : 1.f; }
 struct GroupBufs {
   size_t X[2];
   size_t nb[4];
+  size_t part, part_bytes;
 };
 
 size_t layout_group(int64_t rows, int64_t cols, int count, Op t, const muon_ns_params* p, size_t off,
@@ -83,7 +84,12 @@ size_t layout_group(int64_t rows, int64_t cols, int count, Op t, const muon_ns_p
     if (b) b->nb[i] = off;
     off += nbytes;
   }
-  return off;
+  const size_t pb = t == Op::F32 ? 0 : tc_split_scratch(n, rows < cols ? cols : rows, count);
+  if (b) {
+    b->part = off;
+    b->part_bytes = pb;
+  }
+  return off + up(pb);
 }
 
 template <typename T>
@@ -181,6 +187,8 @@ muon_status polar_impl(const void* X, muon_dtype x_dtype, void* O, muon_dtype o_
   g.xscale = at<float>(ws, q.xscale);
   for (int i = 0; i < ns_work_buffers(&pp); ++i) g.nb[i] = at<void>(ws, q.g.nb[i]);
   g.rho = rho_for(t, n);
+  g.part = q.g.part_bytes ? at<float>(ws, q.g.part) : nullptr;
+  g.part_bytes = q.g.part_bytes;
   TRY(ns_run(t, &g, 1, &pp, status, timeout_ns(), s));
   return launch_copy_out(g.X[g.cur], t, pad_ld(cols), O, o_dtype == MUON_F32 ? Op::F32 : Op::BF16, rows, cols, s);
 }
@@ -398,6 +406,8 @@ muon_status step_impl(const muon_matrix* mats, int32_t count, const muon_params*
     n.cur = 0;
     for (int k = 0; k < ns_work_buffers(&p->ns); ++k) n.nb[k] = at<void>(ws, g.b.nb[k]);
     n.rho = rho_for(t, g.rows < g.cols ? g.rows : g.cols);
+    n.part = g.b.part_bytes ? at<float>(ws, g.b.part) : nullptr;
+    n.part_bytes = g.b.part_bytes;
   }
   for (size_t gi = 0; gi < q.groups.size(); ++gi) ns[gi].xscale = xs + q.groups[gi].slot0;
   E.mark(1, s);

@@ -59,6 +59,19 @@ template <> struct Elem<__half> {
 };
 
 // ---------------------------------------------------------------------------
+// programmatic dependent launch
+// ---------------------------------------------------------------------------
+
+// Wait until the grids this launch depends on have completed and their
+// memory is visible (returns at once for a launch without that attribute).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the next launch in the stream to start its prologue; its own
+// grid_dependency_wait still orders it after this grid's completion.
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // warp / block reductions (fixed order: deterministic)
 // ---------------------------------------------------------------------------
 

@@ -31,6 +31,14 @@
 // triangular scheduler over lower tiles and a transposed-tile epilogue) are
 // scheduled over the tiles that touch the lower triangle only.
 //
+// Split K: a symmetric launch with fewer tiles than the GPU has CTAs (or
+// pairs), e.g. X X^T of a 2048-row matrix with K = 16384, may split each
+// tile's K range into `splits` contiguous parts, one work unit each. Such a
+// unit stores its raw fp32 accumulator (lower sub-tiles only) to a partial
+// buffer, and split_reduce_kernel then sums the parts in a fixed order,
+// applies the epilogue and writes the direct and mirrored copies, so the
+// result is deterministic and exactly symmetric.
+//
 // Every wait is bounded (mbar_wait_bounded): on expiry the kernel records
 // MUON_ERR_TIMEOUT, every role stops, in-flight copies and MMAs are drained
 // with bounded waits and TMEM is freed before the CTA exits.
@@ -74,6 +82,7 @@ struct Group {
   CUtensorMap tmA;
   CUtensorMap tmB;
   CUtensorMap tmD;  // 32x32 boxes, 64-byte swizzle: epilogue stores
+  CUtensorMap tmP;  // split K: fp32 partials [splits*batch][M][ldp], 32x32 boxes, 128-byte swizzle
   void* D;
   const void* C;
   const float* scale;
@@ -82,7 +91,8 @@ struct Group {
   int a_mn, b_mn, sym;
   int alpha_pow, beta_pow;
   float alpha, beta, gamma;
-  int tiles_m, tiles_n, tiles_per_batch, tile_begin;
+  int tiles_m, tiles_n, tiles_per_batch, tile_begin;  // tiles_per_batch counts (tile, split) units
+  int splits, kbps;                                    // K split in parts of kbps k-blocks (1, all)
 };
 
 struct Params {
@@ -95,6 +105,8 @@ struct Params {
 
 struct Tile {
   int g, b, m0, n0;  // m0: first row of the (pair) tile
+  int kb0, kb1;      // k-blocks [kb0, kb1) of this work unit
+  int split;
 };
 
 // Tiles of row block i (tile_m rows) that touch the lower triangle.
@@ -111,6 +123,8 @@ __device__ inline Tile decode(const Params& p, int tile) {
   int local = tile - g.tile_begin;
   int b = local / g.tiles_per_batch;
   int t = local - b * g.tiles_per_batch;
+  const int split = t % g.splits;  // the parts of one tile run side by side
+  t /= g.splits;
   int tm, tn;
   if (!g.sym) {
     tm = t % g.tiles_m;  // M fastest: concurrent CTAs share the B column block
@@ -126,7 +140,10 @@ __device__ inline Tile decode(const Params& p, int tile) {
     tm = i;
     tn = t;
   }
-  return Tile{gi, b, tm * Cfg<PAIR>::TILE_M, tn * BN};
+  const int nkb = (g.K + BK - 1) / BK;
+  const int kb0 = split * g.kbps;
+  const int kb1 = kb0 + g.kbps < nkb ? kb0 + g.kbps : nkb;
+  return Tile{gi, b, tm * Cfg<PAIR>::TILE_M, tn * BN, kb0, kb1, split};
 }
 
 __device__ __forceinline__ float powi(float s, int p) {
@@ -213,12 +230,17 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       prefetch_tmap(&p.g[i].tmA);
       prefetch_tmap(&p.g[i].tmB);
       prefetch_tmap(&p.g[i].tmD);
+      if (p.g[i].splits > 1) prefetch_tmap(&p.g[i].tmP);
     }
   }
   tc_fence_before();
   __syncwarp();
   if (PAIR == 2) cluster_sync(); else __syncthreads();  // barriers initialised in both CTAs
   tc_fence_after();
+  // The setup above overlaps the previous launch's tail; its outputs are
+  // read (and the buffers it reads overwritten) only after this point.
+  grid_dependency_wait();
+  grid_dependents_launch();
   const uint32_t tmem_base = *tmem_slot;
   const uint64_t budget = p.timeout_ns;
 
@@ -238,11 +260,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     for (int tile = unit; tile < p.total_tiles; tile += units) {
       const Tile t = decode<PAIR>(p, tile);
       const Group& g = p.g[t.g];
-      const int nkb = (g.K + BK - 1) / BK;
       const int am0 = t.m0 + (int)rank * BM;            // this CTA's rows of A
       const int bn0 = t.n0 + (int)rank * (BN / PAIR);   // this CTA's rows of B
       bool ok = true;
-      for (int kb = 0; kb < nkb; ++kb) {
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
         if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, budget, p.status)) {
           ok = false;
           break;
@@ -309,7 +330,6 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     for (int tile = unit; tile < p.total_tiles && ok; tile += units) {
       const Tile t = decode<PAIR>(p, tile);
       const Group& g = p.g[t.g];
-      const int nkb = (g.K + BK - 1) / BK;
       const uint32_t idesc = idesc_f16(fmt, g.a_mn, g.b_mn, BM * PAIR, BN);
       // K-major: 8-row groups 1024 B apart, one K step = 32 B inside the
       // swizzle atom. MN-major: 64-element MN atoms 8 KB apart (LBO), 8-row
@@ -319,7 +339,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, budget, p.status)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * BN;
-      for (int kb = 0; kb < nkb; ++kb) {
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
         if (!mbar_wait_bounded(&full[stage], phase, abort_flag, budget, p.status)) {
           ok = false;
           break;
@@ -330,8 +350,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         for (int k = 0; k < BK / UMMA_K; ++k) {
           const uint64_t ad = smem_desc_sw128(a_addr + k * a_kstep, a_lbo, 1024);
           const uint64_t bd = smem_desc_sw128(b_addr + k * b_kstep, b_lbo, 1024);
-          if (PAIR == 2) umma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0);
-          else umma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          const bool accumulate = kb != t.kb0 || k != 0;
+          if (PAIR == 2) umma_f16_pair(d_tmem, ad, bd, idesc, accumulate);
+          else umma_f16(d_tmem, ad, bd, idesc, accumulate);
         }
         // frees the stage (in both CTAs) once these MMAs have read it
         if (PAIR == 2) umma_commit_pair(&empty[stage], 0x3); else umma_commit(&empty[stage]);
@@ -381,18 +402,26 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       const int r0 = t.m0 + (int)rank * BM + q * 32;
       const int row = r0 + lane;
       const int cbase = t.n0 + half * (BN / 2);
-      // The C rows this thread needs, loaded for all its chunks before the
-      // first TMEM read so their latency overlaps instead of adding up.
+      // The C blocks of all its chunks, loaded before the first TMEM read so
+      // their latency overlaps instead of adding up. Loads are coalesced:
+      // load j of a chunk covers block rows 8j..8j+7, four lanes per 64-byte
+      // row; the block is handed to lane = row through shared memory later.
       uint4 cv[EPI_CHUNKS][4];
-      const bool want_c = g.beta != 0.f && row < g.M;
+      const bool part = g.splits > 1;  // store the raw fp32 partial accumulator
+      const bool want_c = g.beta != 0.f && !part;  // warp-uniform
       if (want_c) {
-        const T* c = reinterpret_cast<const T*>(g.C) + (long long)t.b * g.sC + (long long)row * g.ldc + cbase;
+        const T* cb = reinterpret_cast<const T*>(g.C) + (long long)t.b * g.sC + (lane & 3) * 8;
 #pragma unroll
-        for (int ch = 0; ch < EPI_CHUNKS; ++ch)
-          if (cbase + ch * 32 < g.N) {
+        for (int ch = 0; ch < EPI_CHUNKS; ++ch) {
+          const int c0 = cbase + ch * 32;
+          if (c0 < g.N && !(g.sym && c0 > r0 + 31)) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) cv[ch][j] = *reinterpret_cast<const uint4*>(c + ch * 32 + j * 8);
+            for (int j = 0; j < 4; ++j) {
+              const int cr = r0 + 8 * j + (lane >> 2);
+              if (cr < g.M) cv[ch][j] = *reinterpret_cast<const uint4*>(cb + (long long)cr * g.ldc + c0);
+            }
           }
+        }
       }
 #pragma unroll
       for (int ch = 0; ch < EPI_CHUNKS; ++ch) {
@@ -402,19 +431,45 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         uint32_t raw[32];
         tmem_ld_32x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + half * (BN / 2) + ch * 32, raw);
         tmem_wait_ld();
+        if (part) {
+          // 32 fp32 of row `lane` fill one 128-byte row of the staged block
+          // (128-byte swizzle: 16-byte chunk index XOR row % 8)
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<uint4*>(sd + lane * 128 + ((k ^ (lane & 7)) << 4)) =
+                make_uint4(raw[4 * k], raw[4 * k + 1], raw[4 * k + 2], raw[4 * k + 3]);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&g.tmP, smem_u32(sd), c0, r0, t.split * g.batch + t.b);
+            bulk_commit();
+          }
+          continue;
+        }
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = alpha * __uint_as_float(raw[j]);
+        // the previous chunk's bulk stores must have finished reading the staging blocks
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
         if (want_c) {
+          // C block through the mirror staging block (64-byte swizzle):
+          // written as loaded, read back as this lane's row
+#pragma unroll
+          for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(sm + sw64(8 * j + (lane >> 2), (lane & 3) * 8)) = cv[ch][j];
+          __syncwarp();
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const uint4 u = cv[ch][j];
+            const uint4 u = *reinterpret_cast<const uint4*>(sm + sw64(lane, 8 * j));
             float2 f;
             f = Elem<T>::unpack2(u.x); v[8 * j] += beta * f.x; v[8 * j + 1] += beta * f.y;
             f = Elem<T>::unpack2(u.y); v[8 * j + 2] += beta * f.x; v[8 * j + 3] += beta * f.y;
             f = Elem<T>::unpack2(u.z); v[8 * j + 4] += beta * f.x; v[8 * j + 5] += beta * f.y;
             f = Elem<T>::unpack2(u.w); v[8 * j + 6] += beta * f.x; v[8 * j + 7] += beta * f.y;
           }
+          __syncwarp();  // every lane has its row before the block is overwritten
         }
         if (g.gamma != 0.f) {
           const int j = row - c0;
@@ -431,9 +486,6 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         for (int j = 0; j < 16; ++j) pk[j] = Elem<T>::pack2(v[2 * j], v[2 * j + 1]);
         const bool diag = g.sym && c0 == r0;   // the block straddles the diagonal
         const bool mirror = g.sym && r0 > c0;  // strictly lower: also store its transpose
-        // the previous chunk's bulk stores must have finished reading the staging blocks
-        if (lane == 0) bulk_wait_read0();
-        __syncwarp();
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           *reinterpret_cast<uint4*>(sd + sw64(lane, 8 * k)) =
@@ -484,6 +536,107 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
   }
 }
 
+// ---------------------------------------------------------------------------
+// Split-K reduction: D = alpha*s^alpha_pow*sum_parts + beta*s^beta_pow*C +
+// gamma*I over the lower triangle of symmetric n x n outputs, parts summed in
+// increasing order; each 32x32 lower block is written at its place and, off
+// the diagonal, transposed at the mirrored place (a diagonal block takes its
+// upper half from its lower half), so D is exactly symmetric.
+// ---------------------------------------------------------------------------
+
+struct SplitGroup {
+  const float* part;  // [splits][batch][n][ldp]
+  void* D;
+  const void* C;
+  const float* scale;
+  long long ldp, ldd, sD, ldc, sC;
+  int n, batch, splits, nb32, blocks_per_batch, block_begin;
+  int alpha_pow, beta_pow;
+  float alpha, beta, gamma;
+};
+
+struct SplitParams {
+  SplitGroup g[kMaxGemmGroups];
+  int ngroups;
+};
+
+constexpr int RED_THREADS = 256;  // one 32x32 block: 32 rows x 8 groups of 4 columns
+constexpr int RED_MAX_PARTS = 8;
+
+template <typename T>
+__global__ void __launch_bounds__(RED_THREADS) split_reduce_kernel(const __grid_constant__ SplitParams p) {
+  __shared__ float tile[32][33];
+  grid_dependency_wait();
+  int gi = 0;
+  while (gi + 1 < p.ngroups && (int)blockIdx.x >= p.g[gi + 1].block_begin) ++gi;
+  const SplitGroup& g = p.g[gi];
+  const int local = (int)blockIdx.x - g.block_begin;
+  const int b = local / g.blocks_per_batch;
+  const int k = local - b * g.blocks_per_batch;
+  // lower-triangle block k, row by row: (bi, bj) with bj <= bi
+  int bi = (int)((sqrtf(8.f * (float)k + 1.f) - 1.f) * 0.5f);
+  while (bi * (bi + 1) / 2 > k) --bi;
+  while ((bi + 1) * (bi + 2) / 2 <= k) ++bi;
+  const int bj = k - bi * (bi + 1) / 2;
+  const int rr = threadIdx.x >> 3, cg = (threadIdx.x & 7) * 4;  // this thread: row rr, columns cg..cg+3
+  const int r = bi * 32 + rr, c = bj * 32 + cg;
+  float v[4] = {0.f, 0.f, 0.f, 0.f};
+  if (r < g.n) {
+    // every part's 4 values in flight at once (the rows' padding keeps the
+    // 16-byte loads inside the buffer); then summed in part order
+    const float* pp = g.part + ((long long)b * g.n + r) * g.ldp + c;
+    const long long pstride = (long long)g.batch * g.n * g.ldp;
+    float4 pv[RED_MAX_PARTS];
+#pragma unroll
+    for (int sp = 0; sp < RED_MAX_PARTS; ++sp)
+      if (sp < g.splits) pv[sp] = *reinterpret_cast<const float4*>(pp + sp * pstride);
+    float4 acc = pv[0];
+#pragma unroll
+    for (int sp = 1; sp < RED_MAX_PARTS; ++sp)
+      if (sp < g.splits) {
+        acc.x += pv[sp].x;
+        acc.y += pv[sp].y;
+        acc.z += pv[sp].z;
+        acc.w += pv[sp].w;
+      }
+    const float sc = g.scale ? g.scale[b] : 1.f;
+    const float alpha = g.alpha * powi(sc, g.alpha_pow);
+    const float beta = g.beta * powi(sc, g.beta_pow);
+    v[0] = alpha * acc.x;
+    v[1] = alpha * acc.y;
+    v[2] = alpha * acc.z;
+    v[3] = alpha * acc.w;
+    if (g.beta != 0.f) {
+      const T* cr = reinterpret_cast<const T*>(g.C) + (long long)b * g.sC + (long long)r * g.ldc + c;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[j] += beta * Elem<T>::to_f(cr[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (r == c + j) v[j] += g.gamma;
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) tile[rr][cg + j] = Elem<T>::to_f(Elem<T>::from_f(v[j]));  // rounded once
+  __syncthreads();
+  T* D = reinterpret_cast<T*>(g.D) + (long long)b * g.sD;
+  if (r < g.n) {
+    // direct block; a diagonal block takes its upper half from its lower half
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int cc = cg + j;
+      const float x = (bi == bj && cc > rr) ? tile[cc][rr] : tile[rr][cc];
+      if (c + j < g.n) D[(long long)r * g.ldd + c + j] = Elem<T>::from_f(x);
+    }
+  }
+  if (bi != bj) {
+    // mirrored block: D[bj*32 + rr][bi*32 + cg + j] = value at (bi*32 + cg + j, bj*32 + rr)
+    const int rm = bj * 32 + rr, cm = bi * 32 + cg;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (rm < g.n && cm + j < g.n) D[(long long)rm * g.ldd + cm + j] = Elem<T>::from_f(tile[cg + j][rr]);
+  }
+}
+
 }  // namespace tc
 
 // ---------------------------------------------------------------------------
@@ -517,9 +670,12 @@ bool make_map(CUtensorMap* m, Op t, const void* base, int64_t inner, int64_t out
               CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  const CUtensorMapDataType dt = t == Op::BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUtensorMapDataType dt = t == Op::BF16  ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                 : t == Op::F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const cuuint64_t es = op_size(t);
   cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)outer, (cuuint64_t)batch};
-  cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)(batch > 1 ? bstride : ld * outer) * 2};
+  cuuint64_t strides[2] = {(cuuint64_t)ld * es, (cuuint64_t)(batch > 1 ? bstride : ld * outer) * es};
   cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
@@ -527,20 +683,22 @@ bool make_map(CUtensorMap* m, Op t, const void* base, int64_t inner, int64_t out
   return r == CUDA_SUCCESS;
 }
 
+// Co-resident CTAs (PAIR = 1) or clusters (PAIR = 2) of the persistent
+// kernel; 0 if its attributes cannot be set.
 template <typename T, int PAIR>
-muon_status launch(const tc::Params& p, int total_tiles, cudaStream_t s) {
+int max_units() {
   static bool attr_set = false;
-  static int max_units = 0;  // co-resident CTAs (PAIR = 1) or clusters (PAIR = 2)
+  static int units = 0;
   const void* fn = (const void*)tc::gemm_kernel<T, PAIR>;
   if (!attr_set) {
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Cfg<PAIR>::SMEM) != cudaSuccess)
-      return MUON_ERR_CUDA;
-    max_units = num_sms() / PAIR;
+      return 0;
+    units = num_sms() / PAIR;
     if (PAIR == 2) {
       // not every SM may have a free partner in its GPC: launch only as many
       // persistent pairs as can run at once
       cudaLaunchConfig_t q = {};
-      q.gridDim = dim3(2 * max_units);
+      q.gridDim = dim3(2 * units);
       q.blockDim = dim3(tc::THREADS);
       q.dynamicSmemBytes = tc::Cfg<PAIR>::SMEM;
       cudaLaunchAttribute a[1];
@@ -551,29 +709,79 @@ muon_status launch(const tc::Params& p, int total_tiles, cudaStream_t s) {
       q.attrs = a;
       q.numAttrs = 1;
       int clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&clusters, fn, &q) == cudaSuccess && clusters > 0 && clusters < max_units)
-        max_units = clusters;
+      if (cudaOccupancyMaxActiveClusters(&clusters, fn, &q) == cudaSuccess && clusters > 0 && clusters < units)
+        units = clusters;
       cudaGetLastError();
     }
     attr_set = true;
   }
+  return units;
+}
+
+template <typename T, int PAIR>
+muon_status launch(const tc::Params& p, int total_tiles, int max_units, cudaStream_t s) {
   const int units = total_tiles < max_units ? total_tiles : max_units;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(units * PAIR);
   cfg.blockDim = dim3(tc::THREADS);
   cfg.dynamicSmemBytes = tc::Cfg<PAIR>::SMEM;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = PAIR;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, tc::gemm_kernel<T, PAIR>, p) == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
 }
 
+template <typename T>
+muon_status launch_reduce(const tc::SplitParams& p, int blocks, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(tc::RED_THREADS);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc::split_reduce_kernel<T>, p) == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
+}
+
 int g_pair_mode = 2;  // 2: CTA-pair kernel, 1: single-CTA kernel
+
+// Split K only while every part keeps at least kMinSplitKb k-blocks (64 K
+// each), so the partial traffic stays small against the part's MMAs.
+constexpr int kMaxSplits = 8;
+static_assert(kMaxSplits <= tc::RED_MAX_PARTS, "the reduction holds every part in registers");
+constexpr int kMinSplitKb = 32;
+
+int sym_tiles(int64_t n, int tile_m) {
+  const int tm = (int)((n + tile_m - 1) / tile_m), tn = (int)((n + tc::BN - 1) / tc::BN);
+  int c = 0;
+  for (int i = 0; i < tm; ++i) c += tc::sym_row_tiles(i, tn, tile_m);
+  return c;
+}
+
+// Parts for a symmetric launch of `tiles` tiles over `units` CTAs (pairs)
+// with nkb k-blocks per tile; sets *kbps to the k-blocks per part.
+int split_parts(int tiles, int units, int nkb, int* kbps) {
+  *kbps = nkb;
+  if (tiles <= 0 || tiles >= units) return 1;
+  int want = units / tiles;
+  if (want > kMaxSplits) want = kMaxSplits;
+  if (want < 2) return 1;
+  int per = (nkb + want - 1) / want;
+  if (per < kMinSplitKb) per = kMinSplitKb;
+  const int parts = (nkb + per - 1) / per;  // every part has at least one k-block
+  if (parts < 2) return 1;
+  *kbps = per;
+  return parts;
+}
 
 }  // namespace
 
@@ -589,13 +797,34 @@ int num_sms() {
 
 void set_gemm_pair_mode(int pair) { g_pair_mode = pair == 1 ? 1 : 2; }
 
+size_t tc_split_scratch(int64_t n, int64_t K, int count) {
+  size_t best = 0;
+  const int nkb = (int)((K + tc::BK - 1) / tc::BK);
+  for (int pair = 1; pair <= 2; ++pair) {
+    // num_sms() / pair bounds the co-resident units from above, so the
+    // reservation covers every launch this group takes part in
+    int kbps = 0;
+    const int parts = split_parts(count * sym_tiles(n, tc::BM * pair), num_sms() / pair, nkb, &kbps);
+    if (parts > 1) {
+      const size_t b = (size_t)parts * count * n * pad_ld(n) * sizeof(float);
+      if (b > best) best = b;
+    }
+  }
+  return best;
+}
+
 muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t timeout_ns, cudaStream_t s) {
   if (ngroups < 1 || ngroups > kMaxGemmGroups || (t != Op::BF16 && t != Op::F16)) return MUON_ERR_INVALID_ARG;
   const int pair = g_pair_mode;
   const int tile_m = tc::BM * pair;
+  const int units = pair == 2 ? (t == Op::BF16 ? max_units<__nv_bfloat16, 2>() : max_units<__half, 2>())
+                              : (t == Op::BF16 ? max_units<__nv_bfloat16, 1>() : max_units<__half, 1>());
+  if (units <= 0) return MUON_ERR_CUDA;
   tc::Params p;
   memset(&p, 0, sizeof(p));
-  int total = 0;
+  const GemmDesc* src[kMaxGemmGroups];
+  int base_tiles[kMaxGemmGroups];
+  int total_base = 0;
   int ng = 0;
   for (int i = 0; i < ngroups; ++i) {
     const GemmDesc& d = gd[i];
@@ -632,36 +861,88 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
     g.gamma = d.gamma;
     g.tiles_m = (d.M + tile_m - 1) / tile_m;
     g.tiles_n = (d.N + tc::BN - 1) / tc::BN;
-    if (d.sym) {
-      int c = 0;
-      for (int i2 = 0; i2 < g.tiles_m; ++i2) c += tc::sym_row_tiles(i2, g.tiles_n, tile_m);
-      g.tiles_per_batch = c;
-    } else {
-      g.tiles_per_batch = g.tiles_m * g.tiles_n;
-    }
-    g.tile_begin = total;
-    total += g.tiles_per_batch * d.batch;
+    g.tiles_per_batch = d.sym ? sym_tiles(d.M, tile_m) : g.tiles_m * g.tiles_n;
+    g.splits = 1;
+    g.kbps = (d.K + tc::BK - 1) / tc::BK;
+    src[ng] = &d;
+    base_tiles[ng] = g.tiles_per_batch;
+    total_base += g.tiles_per_batch * d.batch;
     ++ng;
   }
   if (ng == 0) return MUON_OK;
+
+  // split K where the launch leaves CTAs (pairs) idle and a scratch is given
+  tc::SplitParams sp;
+  memset(&sp, 0, sizeof(sp));
+  int red_blocks = 0;
+  for (int i = 0; i < ng; ++i) {
+    tc::Group& g = p.g[i];
+    const GemmDesc& d = *src[i];
+    if (!d.sym || !d.part) continue;
+    int kbps = 0;
+    const int parts = split_parts(total_base, units, g.kbps, &kbps);
+    const int64_t ldp = pad_ld(d.N);
+    if (parts < 2 || (size_t)parts * d.batch * d.N * ldp * sizeof(float) > d.part_bytes) continue;
+    if (!make_map(&g.tmP, Op::F32, d.part, d.N, d.M, (int64_t)parts * d.batch, ldp, (int64_t)d.M * ldp, 32, 32))
+      return MUON_ERR_CUDA;
+    g.splits = parts;
+    g.kbps = kbps;
+    g.tiles_per_batch *= parts;
+    tc::SplitGroup& r = sp.g[sp.ngroups++];
+    r.part = d.part;
+    r.D = d.D;
+    r.C = d.C;
+    r.scale = d.scale;
+    r.ldp = ldp;
+    r.ldd = d.ldd;
+    r.sD = d.strideD;
+    r.ldc = d.ldc;
+    r.sC = d.strideC;
+    r.n = d.N;
+    r.batch = d.batch;
+    r.splits = parts;
+    r.nb32 = (d.N + 31) / 32;
+    r.blocks_per_batch = r.nb32 * (r.nb32 + 1) / 2;
+    r.block_begin = red_blocks;
+    r.alpha_pow = d.alpha_pow;
+    r.beta_pow = d.beta_pow;
+    r.alpha = d.alpha;
+    r.beta = d.beta;
+    r.gamma = d.gamma;
+    red_blocks += r.blocks_per_batch * d.batch;
+    // the GEMM stores raw accumulators; the reduction applies the epilogue
+    g.alpha = 1.f;
+    g.alpha_pow = 0;
+    g.beta = 0.f;
+    g.gamma = 0.f;
+  }
+  int total = 0;
+  for (int i = 0; i < ng; ++i) {
+    p.g[i].tile_begin = total;
+    total += p.g[i].tiles_per_batch * p.g[i].batch;
+  }
   p.ngroups = ng;
   p.total_tiles = total;
   p.status = status;
   p.timeout_ns = timeout_ns;
 
   Counters& cn = counters();
-  cn.launches += 1;
+  cn.launches += sp.ngroups ? 2 : 1;
   cn.gemm_launches += 1;
   for (int i = 0; i < ng; ++i) {
     const tc::Group& g = p.g[i];
     const double mnk = (double)g.M * g.N * g.K * g.batch;
     cn.flops_dense += 2.0 * mnk;
     cn.flops_sym += g.sym ? mnk : 2.0 * mnk;
-    cn.flops_exec += 2.0 * tile_m * tc::BN * (double)g.K * g.tiles_per_batch * g.batch;
+    cn.flops_exec += 2.0 * tile_m * tc::BN * (double)g.K * base_tiles[i] * g.batch;
   }
+  muon_status r;
   if (pair == 2)
-    return t == Op::BF16 ? launch<__nv_bfloat16, 2>(p, total, s) : launch<__half, 2>(p, total, s);
-  return t == Op::BF16 ? launch<__nv_bfloat16, 1>(p, total, s) : launch<__half, 1>(p, total, s);
+    r = t == Op::BF16 ? launch<__nv_bfloat16, 2>(p, total, units, s) : launch<__half, 2>(p, total, units, s);
+  else
+    r = t == Op::BF16 ? launch<__nv_bfloat16, 1>(p, total, units, s) : launch<__half, 1>(p, total, units, s);
+  if (r != MUON_OK || sp.ngroups == 0) return r;
+  return t == Op::BF16 ? launch_reduce<__nv_bfloat16>(sp, red_blocks, s) : launch_reduce<__half>(sp, red_blocks, s);
 }
 
 }  // namespace muon

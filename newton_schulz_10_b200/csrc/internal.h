@@ -29,6 +29,7 @@ inline int64_t pad_ld(int64_t cols) { return (cols + 63) / 64 * 64; }
 //   D = alpha*s^alpha_pow*acc + beta*s^beta_pow*C + gamma*I, s = scale[b]
 //   (s = 1 when scale is NULL); sym = 1: M == N and D is symmetric: only the
 //   lower triangle is computed and mirrored (D is then exactly symmetric).
+//   part: optional fp32 scratch of part_bytes for split K (symmetric only).
 struct GemmDesc {
   const void* A;
   int64_t lda, strideA;
@@ -43,11 +44,20 @@ struct GemmDesc {
   float alpha, beta, gamma;
   const float* scale;
   int alpha_pow, beta_pow;
+  float* part;
+  size_t part_bytes;
 };
 
 // Tensor-core GEMM (tcgen05 + TMEM + TMA), all groups in one persistent launch.
 // Operand type bf16 or f16. Returns MUON_OK or MUON_ERR_CUDA.
+// A symmetric launch with fewer tiles than CTAs (pairs) splits K over the
+// `part` scratch when it is large enough, then reduces the parts in a second
+// launch.
 muon_status tc_gemm(Op t, const GemmDesc* g, int ngroups, int* status, uint64_t timeout_ns, cudaStream_t s);
+
+// Bytes of split-K scratch that X X^T (n x n, inner dimension K) of a group
+// of `count` matrices can use in any launch; 0 when it never splits.
+size_t tc_split_scratch(int64_t n, int64_t K, int count);
 
 // fp32 FFMA GEMM (no TF32), one group per launch.
 muon_status simt_gemm(const GemmDesc& g, cudaStream_t s);
@@ -74,6 +84,7 @@ Counters& counters();
 //   nb[]         [count][n][ldn] work matrices, n = min(rows, cols),
 //                ldn = pad_ld(n): 2 for the standard chain, 4 for Gram
 //   rho          Gram only: R is stored as rho * X X^T (keeps fp16 in range)
+//   part         split-K scratch of the X X^T products (NULL: no split)
 struct NsGroup {
   int64_t rows, cols;
   int count;
@@ -82,6 +93,8 @@ struct NsGroup {
   const float* xscale;
   void* nb[4];
   float rho;
+  float* part;
+  size_t part_bytes;
 };
 
 inline int ns_work_buffers(const muon_ns_params* p) { return p->gram ? 4 : 2; }

@@ -57,6 +57,8 @@ GemmDesc gram_of(const NsGroup& g, const void* X, void* D, float alpha, const fl
   d.alpha = alpha;
   d.scale = scale;
   d.alpha_pow = apow;
+  d.part = g.part;
+  d.part_bytes = g.part_bytes;
   return d;
 }
 
@@ -75,6 +77,8 @@ GemmDesc sym_of(const NsGroup& g, const void* P, const void* Q, void* D, const v
   d.alpha = alpha;
   d.beta = beta;
   d.gamma = gamma;
+  d.part = g.part;
+  d.part_bytes = g.part_bytes;
   return d;
 }
 

@@ -12,7 +12,7 @@ namespace muon {
 namespace {
 
 constexpr int BLOCK = 256;
-constexpr int UNROLL = 4;  // momentum pass: 16-byte vectors of M and G in flight per lane
+constexpr int UNROLL = 4;  // 16-byte vectors in flight per lane (momentum, row statistics, copy-out)
 
 __device__ __forceinline__ int find_mat(const RowLaunch& L, int task) {
   int lo = 0, hi = L.count - 1;
@@ -159,12 +159,22 @@ __global__ void __launch_bounds__(BLOCK) row_stats(const __grid_constant__ RowLa
   if (active) {
     const S* x = reinterpret_cast<const S*>(m.src) + r * m.cols;
     if ((m.cols & 3) == 0) {
-      for (int64_t c = l; c < (m.cols >> 2); c += WG) {
-        const float4 v = Src<S>::load4(x + 4 * c);
+      const int64_t n4 = m.cols >> 2;
+      auto add = [&](const float4 v) {
         const double a = v.x, b = v.y, cc = v.z, d = v.w;
         ss += a * a + b * b + cc * cc + d * d;
         sa += fabs(a) + fabs(b) + fabs(cc) + fabs(d);
+      };
+      int64_t c = l;
+      // UNROLL vectors in flight per lane; summed in the same order as one at a time
+      for (; c + (UNROLL - 1) * WG < n4; c += UNROLL * WG) {
+        float4 v[UNROLL];
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) v[u] = Src<S>::load4(x + 4 * (c + u * WG));
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) add(v[u]);
       }
+      for (; c < n4; c += WG) add(Src<S>::load4(x + 4 * c));
     } else {
       for (int64_t c = l; c < m.cols; c += WG) {
         const double a = Src<S>::load1(x + c);
@@ -451,6 +461,32 @@ __device__ void normuon_finalize_block(float* rscale, int64_t k, int64_t m, floa
   for (int64_t i = threadIdx.x; i < k; i += BLOCK) rscale[i] = ratio * rscale[i];
 }
 
+// cols % 4 == 0: vectors of 4, UNROLL of them in flight per thread
+template <typename I, typename O>
+__global__ void __launch_bounds__(BLOCK) copy_out4(const I* in, int64_t ldi, O* out, int64_t rows, int64_t cols) {
+  const int64_t n4 = cols >> 2, total = rows * n4;
+  const int64_t stride = (int64_t)gridDim.x * BLOCK;
+  for (int64_t e0 = blockIdx.x * (int64_t)BLOCK + threadIdx.x; e0 < total; e0 += stride * UNROLL) {
+    float4 v[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int64_t e = e0 + u * stride;
+      if (e < total) {
+        const int64_t r = e / n4, c = (e - r * n4) << 2;
+        v[u] = Src<I>::load4(in + r * ldi + c);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int64_t e = e0 + u * stride;
+      if (e < total) {
+        const int64_t r = e / n4, c = (e - r * n4) << 2;
+        Dst<O>::store4(out + r * cols + c, v[u]);
+      }
+    }
+  }
+}
+
 template <typename I, typename O>
 __global__ void __launch_bounds__(BLOCK) copy_out(const I* in, int64_t ldi, O* out, int64_t rows, int64_t cols) {
   const int64_t total = rows * cols;
@@ -623,7 +659,12 @@ muon_status launch_copy_out(const void* in, Op it, int64_t ldi, void* out, Op ot
   if (total == 0) return MUON_OK;
   int64_t g = (total + BLOCK - 1) / BLOCK;
   if (g > 148 * 16) g = 148 * 16;
-#define CP(I, O) copy_out<I, O><<<(int)g, BLOCK, 0, s>>>(reinterpret_cast<const I*>(in), ldi, reinterpret_cast<O*>(out), rows, cols)
+  const bool v4 = (cols & 3) == 0;  // rows of out then start on 16-byte (f32) / 8-byte (bf16) boundaries
+#define CP(I, O)                                                                                             \
+  do {                                                                                                       \
+    if (v4) copy_out4<I, O><<<(int)g, BLOCK, 0, s>>>(reinterpret_cast<const I*>(in), ldi, reinterpret_cast<O*>(out), rows, cols); \
+    else copy_out<I, O><<<(int)g, BLOCK, 0, s>>>(reinterpret_cast<const I*>(in), ldi, reinterpret_cast<O*>(out), rows, cols);     \
+  } while (0)
   if (it == Op::F32) { if (ot == Op::F32) CP(float, float); else CP(float, __nv_bfloat16); }
   else if (it == Op::F16) { if (ot == Op::F32) CP(__half, float); else CP(__half, __nv_bfloat16); }
   else { if (ot == Op::F32) CP(__nv_bfloat16, float); else CP(__nv_bfloat16, __nv_bfloat16); }

@@ -368,3 +368,66 @@ def test_step_many_tiles_mixed_layouts(pair):
     assert st == mu.OK, mu.status_str(st)
     idx = [0, 39, 40, 47, 48, 55]
     check_step([state[i] for i in idx], [got[i] for i in idx], O.StepParams(), TOL16)
+
+
+# ---------------------------------------------------------------------------
+# split K: X X^T launches with fewer tiles than CTAs (pairs) and a long K
+# ---------------------------------------------------------------------------
+
+
+def _launches(fn):
+    n0 = mu.kernel_launch_count()
+    out = fn()
+    torch.cuda.synchronize()
+    return out, mu.kernel_launch_count() - n0
+
+
+@pytest.mark.parametrize("pair", [True, False])
+@pytest.mark.parametrize("shape", [(300, 9000), (9000, 300)])
+def test_split_k_standard_bf16(pair, shape):
+    """n = 300 rows against K = 9000 (ragged in both): X X^T has a handful of
+    tiles, so each is split along K into fp32 partials that a second launch
+    sums in a fixed order. One reduction launch per X X^T (five)."""
+    X = gauss(shape, 9100 + shape[0])
+    short = gauss((shape[0], 1000) if shape[0] < shape[1] else (1000, shape[1]), 9200)
+    mu.set_gemm_cta_pair(pair)
+    try:
+        (Og, ws), n_split = _launches(lambda: mu.ns_polar(dev(X), mu.ns_params(compute=mu.BF16),
+                                                          out_dtype=torch.float32))
+        (_, ws2), n_plain = _launches(lambda: mu.ns_polar(dev(short), mu.ns_params(compute=mu.BF16),
+                                                          out_dtype=torch.float32))
+        # the same input again: bit-identical (fixed-order reduction)
+        Og2, _ = mu.ns_polar(dev(X), mu.ns_params(compute=mu.BF16), out_dtype=torch.float32)
+    finally:
+        mu.set_gemm_cta_pair(True)
+    assert status_of(ws) == mu.OK and status_of(ws2) == mu.OK
+    assert n_split - n_plain == 5
+    assert torch.equal(Og, Og2)
+    assert rel(host(Og), O.newton_schulz(X.astype(np.float64), COEFFS5)) < TOL16
+
+
+@pytest.mark.parametrize("restart", [3, 0])
+def test_split_k_gram_f16(restart):
+    """Gram NS in fp16 on 520 x 4200: X X^T (at the start and at the restart)
+    is split into parts of 32, 32 and 2 k-blocks (a ragged last part)."""
+    X = gauss((520, 4200), 9300)
+    p = mu.ns_params(gram=True, restart_at=restart, compute=mu.F16)
+    (Og, ws), n_split = _launches(lambda: mu.gram_ns_polar(dev(X), p, out_dtype=torch.float32))
+    (_, ws2), n_plain = _launches(lambda: mu.gram_ns_polar(dev(gauss((520, 1000), 9301)), p,
+                                                           out_dtype=torch.float32))
+    assert status_of(ws) == mu.OK and status_of(ws2) == mu.OK
+    assert n_split - n_plain == (2 if restart else 1)
+    want = O.gram_newton_schulz(X.astype(np.float64), COEFFS5, restart_at=restart)
+    assert rel(host(Og), want) < TOL16
+
+
+def test_split_k_dion3_batched_step():
+    """Dion3 (f = 1/4) + NorMuon + Gram fp16 on two 1024 x 8192 matrices: the
+    selected 256 x 8192 pair shares each X X^T launch, split four ways."""
+    state = make_state([(1024, 8192), (1024, 8192)], 9400, m_std=1e-3)
+    p = mu.step_params(ns=mu.ns_params(gram=True, restart_at=3, compute=mu.F16), normuon=True, dion3=True,
+                       frac=(1, 4), select_norm=mu.NORM_L2)
+    got, st = run_step(state, p)
+    assert st == mu.OK
+    k = O.rows_for_fraction(1024, 1, 4)
+    check_step(state, got, O.StepParams(gram=True, restart_at=3, normuon=True, k=k, select_norm="l2"), TOL16)
