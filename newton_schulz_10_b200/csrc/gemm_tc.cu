@@ -391,21 +391,17 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     for (int tile = unit; tile < p.total_tiles; tile += units) {
       const Tile t = decode<PAIR>(p, tile);
       const Group& g = p.g[t.g];
-      // every lane waits; the verdict is made warp-uniform so the warp-wide
-      // tcgen05.ld below never runs with part of the warp gone
-      const bool ok = mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, budget, p.status);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
       const float s = g.scale ? g.scale[t.b] : 1.f;
       const float alpha = g.alpha * powi(s, g.alpha_pow);
       const float beta = g.beta * powi(s, g.beta_pow);
       const int r0 = t.m0 + (int)rank * BM + q * 32;
       const int row = r0 + lane;
       const int cbase = t.n0 + half * (BN / 2);
-      // The C blocks of all its chunks, loaded before the first TMEM read so
-      // their latency overlaps instead of adding up. Loads are coalesced:
-      // load j of a chunk covers block rows 8j..8j+7, four lanes per 64-byte
-      // row; the block is handed to lane = row through shared memory later.
+      // The C blocks of all its chunks (and the scale above) are loaded
+      // before waiting for the accumulator, so their latency overlaps that
+      // wait. Loads are coalesced: load j of a chunk covers block rows
+      // 8j..8j+7, four lanes per 64-byte row; the block is handed to
+      // lane = row through shared memory later.
       uint4 cv[EPI_CHUNKS][4];
       const bool part = g.splits > 1;  // store the raw fp32 partial accumulator
       const bool want_c = g.beta != 0.f && !part;  // warp-uniform
@@ -423,6 +419,11 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
           }
         }
       }
+      // every lane waits; the verdict is made warp-uniform so the warp-wide
+      // tcgen05.ld below never runs with part of the warp gone
+      const bool ok = mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, budget, p.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
 #pragma unroll
       for (int ch = 0; ch < EPI_CHUNKS; ++ch) {
         const int c0 = cbase + ch * 32;
@@ -511,11 +512,12 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
           bulk_commit();
         }
       }
-      // this warp's TMEM reads are done: release the accumulator (to the leader)
+      // this warp's TMEM reads are done: release the accumulator (to the
+      // leader's barrier; the MMAs that overwrite it wait there)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if (PAIR == 2) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+        if (PAIR == 2 && rank != 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[acc]), 0));
         else mbar_arrive(&tempty[acc]);
       }
       if (++acc == 2) {
