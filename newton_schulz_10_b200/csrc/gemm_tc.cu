@@ -419,7 +419,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
           }
         }
       }
-      // every lane waits; the verdict is made warp-uniform so the warp-wide
+      // every lane waits; the result is made warp-uniform so the warp-wide
       // tcgen05.ld below never runs with part of the warp gone
       const bool ok = mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, budget, p.status);
       if (!__all_sync(0xffffffffu, ok)) break;

@@ -24,7 +24,7 @@ Source of every formula: "Dion3: Full-stack orthogonal updates"
   k = ceil(f n), polar of M[S, :], update W[S, :], error feedback
   M <- mu*M_hat + (M - M_hat).
 
-Readings taken where the page is silent (each also listed in the design doc):
+Readings taken where the page is silent:
 
 * Coefficients (a_t, b_t, c_t) are inputs; the workloads use
   (3.4445, -4.7750, 2.0315) for every t.
