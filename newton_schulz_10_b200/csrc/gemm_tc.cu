@@ -395,7 +395,6 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       const float alpha = g.alpha * powi(s, g.alpha_pow);
       const float beta = g.beta * powi(s, g.beta_pow);
       const int r0 = t.m0 + (int)rank * BM + q * 32;
-      const int row = r0 + lane;
       const int cbase = t.n0 + half * (BN / 2);
       // The C blocks of all its chunks (and the scale above) are loaded
       // before waiting for the accumulator, so their latency overlaps that
@@ -429,10 +428,11 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         const int c0 = cbase + ch * 32;
         if (c0 >= g.N) break;                      // warp-uniform
         if (g.sym && c0 > r0 + 31) break;          // whole sub-tile above the diagonal
-        uint32_t raw[32];
-        tmem_ld_32x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + half * (BN / 2) + ch * 32, raw);
-        tmem_wait_ld();
+        const uint32_t tcol = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + half * (BN / 2) + ch * 32;
         if (part) {
+          uint32_t raw[32];
+          tmem_ld_32x32(tcol, raw);
+          tmem_wait_ld();
           // 32 fp32 of row `lane` fill one 128-byte row of the staged block
           // (128-byte swizzle: 16-byte chunk index XOR row % 8)
           if (lane == 0) bulk_wait_read0();
@@ -449,60 +449,85 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
           }
           continue;
         }
+        // The 32x32 block in the m16n8 fragment layout, as two 16-lane
+        // halves: v[16h + r] is element (16h + 8*((r>>1)&1) + lane/4,
+        // 8*(r>>2) + 2*(lane%4) + (r&1)) of the block. 8x8 matrix (h, s, i)
+        // (rows 16h + 8s.., columns 8i..) is v[16h + 4i + 2s], v[16h + 4i + 2s + 1].
         float v[32];
+        {
+          uint32_t f0[16], f1[16];
+          tmem_ld_16x256_x4(tcol, f0);
+          tmem_ld_16x256_x4(tcol + (16u << 16), f1);
+          tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = alpha * __uint_as_float(raw[j]);
+          for (int r = 0; r < 16; ++r) {
+            v[r] = alpha * __uint_as_float(f0[r]);
+            v[16 + r] = alpha * __uint_as_float(f1[r]);
+          }
+        }
         // the previous chunk's bulk stores must have finished reading the staging blocks
         if (lane == 0) bulk_wait_read0();
         __syncwarp();
+        const uint32_t sd_a = smem_u32(sd), sm_a = smem_u32(sm);
         if (want_c) {
           // C block through the mirror staging block (64-byte swizzle):
-          // written as loaded, read back as this lane's row
+          // written as loaded, read back in the fragment layout
 #pragma unroll
           for (int j = 0; j < 4; ++j) *reinterpret_cast<uint4*>(sm + sw64(8 * j + (lane >> 2), (lane & 3) * 8)) = cv[ch][j];
           __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint4 u = *reinterpret_cast<const uint4*>(sm + sw64(lane, 8 * j));
-            float2 f;
-            f = Elem<T>::unpack2(u.x); v[8 * j] += beta * f.x; v[8 * j + 1] += beta * f.y;
-            f = Elem<T>::unpack2(u.y); v[8 * j + 2] += beta * f.x; v[8 * j + 3] += beta * f.y;
-            f = Elem<T>::unpack2(u.z); v[8 * j + 4] += beta * f.x; v[8 * j + 5] += beta * f.y;
-            f = Elem<T>::unpack2(u.w); v[8 * j + 6] += beta * f.x; v[8 * j + 7] += beta * f.y;
+          for (int k = 0; k < 4; ++k) {  // k = 2h + s
+            uint32_t cf[4];
+            ldsm_x4(sm_a + sw64(16 * (k >> 1) + 8 * (k & 1) + (lane & 7), 8 * (lane >> 3)), cf);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = Elem<T>::unpack2(cf[i]);
+              const int x = 16 * (k >> 1) + 4 * i + 2 * (k & 1);
+              v[x] += beta * f.x;
+              v[x + 1] += beta * f.y;
+            }
           }
-          __syncwarp();  // every lane has its row before the block is overwritten
+          __syncwarp();  // the C block is read before the staging block is overwritten
         }
         if (g.gamma != 0.f) {
-          const int j = row - c0;
-          if (j >= 0 && j < 32) {
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj)
-              if (jj == j) v[jj] += g.gamma;
+          for (int x = 0; x < 32; ++x) {
+            const int rr = 16 * (x >> 4) + 8 * ((x >> 1) & 1) + (lane >> 2);
+            const int cc = 8 * ((x >> 2) & 3) + 2 * (lane & 3) + (x & 1);
+            if (r0 + rr == c0 + cc) v[x] += g.gamma;
           }
         }
         // Round once to the stored type: the direct and mirrored copies of an
         // element are the same bits, so D is exactly symmetric.
-        uint32_t pk[16];
+        uint32_t pk[16];  // pk[4k + i]: matrix (h, s, i) with k = 2h + s
 #pragma unroll
-        for (int j = 0; j < 16; ++j) pk[j] = Elem<T>::pack2(v[2 * j], v[2 * j + 1]);
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int x = 16 * (k >> 1) + 4 * i + 2 * (k & 1);
+            pk[4 * k + i] = Elem<T>::pack2(v[x], v[x + 1]);
+          }
         const bool diag = g.sym && c0 == r0;   // the block straddles the diagonal
         const bool mirror = g.sym && r0 > c0;  // strictly lower: also store its transpose
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          *reinterpret_cast<uint4*>(sd + sw64(lane, 8 * k)) =
-              make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+          stsm_x4(sd_a + sw64(16 * (k >> 1) + 8 * (k & 1) + (lane & 7), 8 * (lane >> 3)), pk[4 * k], pk[4 * k + 1],
+                  pk[4 * k + 2], pk[4 * k + 3]);
+        if (diag || mirror) {
+          // the transposed block: matrix (h, s, i) lands at rows 8i.., columns 16h + 8s..
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            stsm_x4_trans(sm_a + sw64(lane, 16 * (k >> 1) + 8 * (k & 1)), pk[4 * k], pk[4 * k + 1], pk[4 * k + 2],
+                          pk[4 * k + 3]);
+        }
         if (diag) {
-          // symmetrise the diagonal block: above the diagonal (row j < col)
-          // takes the value computed below it, D[j][lane] = D[lane][j]
+          // symmetrise the diagonal block: above the diagonal (row < col)
+          // takes the value computed below it, from the transposed block
           __syncwarp();
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (j < lane) *reinterpret_cast<uint16_t*>(sd + sw64(j, lane)) = (uint16_t)(pk[j >> 1] >> ((j & 1) * 16));
-        }
-        if (mirror) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            *reinterpret_cast<uint16_t*>(sm + sw64(j, lane)) = (uint16_t)(pk[j >> 1] >> ((j & 1) * 16));
+            if (j > lane)
+              *reinterpret_cast<uint16_t*>(sd + sw64(lane, j)) = *reinterpret_cast<const uint16_t*>(sm + sw64(lane, j));
         }
         fence_async_smem();  // generic-proxy writes become visible to the bulk copy
         __syncwarp();
