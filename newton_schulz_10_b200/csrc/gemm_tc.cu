@@ -336,6 +336,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       // K groups 1024 B apart (SBO), one K step of 16 rows = 2048 B.
       const uint32_t a_lbo = g.a_mn ? 8192u : 16u, b_lbo = g.b_mn ? 8192u : 16u;
       const uint32_t a_kstep = g.a_mn ? 2048u : 32u, b_kstep = g.b_mn ? 2048u : 32u;
+      // descriptor fields other than the start address, fixed for the tile;
+      // start addresses (>> 4) stay below 2^14 inside the 228 KB window
+      const uint64_t a_hi = smem_desc_sw128(0, a_lbo, 1024), b_hi = smem_desc_sw128(0, b_lbo, 1024);
       if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, budget, p.status)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * BN;
@@ -344,12 +347,14 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
           ok = false;
           break;
         }
-        tc_fence_after();
-        const uint32_t a_addr = a_base + stage * Cf::A_STAGE, b_addr = b_base + stage * Cf::B_STAGE;
+        // No tcgen05 fence here: the stage barrier completes only when the
+        // copies' bytes have landed, and the MMAs that read them are issued
+        // after the wait returns.
+        const uint32_t a_lo = (a_base + stage * Cf::A_STAGE) >> 4, b_lo = (b_base + stage * Cf::B_STAGE) >> 4;
 #pragma unroll
         for (int k = 0; k < BK / UMMA_K; ++k) {
-          const uint64_t ad = smem_desc_sw128(a_addr + k * a_kstep, a_lbo, 1024);
-          const uint64_t bd = smem_desc_sw128(b_addr + k * b_kstep, b_lbo, 1024);
+          const uint64_t ad = a_hi | (uint64_t)(a_lo + k * (a_kstep >> 4));
+          const uint64_t bd = b_hi | (uint64_t)(b_lo + k * (b_kstep >> 4));
           const bool accumulate = kb != t.kb0 || k != 0;
           if (PAIR == 2) umma_f16_pair(d_tmem, ad, bd, idesc, accumulate);
           else umma_f16(d_tmem, ad, bd, idesc, accumulate);
