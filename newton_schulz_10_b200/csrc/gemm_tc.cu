@@ -53,12 +53,13 @@ namespace muon {
 
 namespace tc {
 
-constexpr int BM = 128, BN = 256, BK = 64;  // BM: rows per CTA
+constexpr int BM = 128, BK = 64;  // BM: rows per CTA
+constexpr int BN_WIDE = 256;      // tile columns: 256, or 128 for launches too small to fill the GPU
+constexpr int BN_NARROW = 128;
 constexpr int UMMA_K = 16;
 constexpr int EPI_WARP0 = 4;
 constexpr int EPI_WARPS = 8;                       // two per TMEM lane quarter
 constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
-constexpr int EPI_CHUNKS = BN / 32 / 2;            // 32-column chunks per epilogue warp
 constexpr int TMEM_COLS = 512;
 constexpr int EPI_BLOCK = 32 * 32 * 2;             // one staged 32x32 block of bf16/fp16, 64-byte rows
 constexpr int EPI_BUF = 2 * EPI_BLOCK;             // per epilogue warp: direct block + mirrored block
@@ -66,11 +67,12 @@ constexpr int EPI_BUF = 2 * EPI_BLOCK;             // per epilogue warp: direct 
 // a tiny configurable wait budget never lets a CTA exit with work in flight.
 constexpr uint64_t DRAIN_NS = 1000000000ull;
 
-template <int PAIR>
+template <int PAIR, int BN>
 struct Cfg {
-  static constexpr int STAGES = PAIR == 2 ? 6 : 4;
+  static constexpr int STAGES = PAIR == 2 ? (BN == BN_WIDE ? 6 : 8) : (BN == BN_WIDE ? 4 : 6);
   static constexpr int A_STAGE = BM * BK * 2;                  // this CTA's 128 rows of A
-  static constexpr int B_STAGE = (BN / PAIR) * BK * 2;         // this CTA's share of B's 256 rows
+  static constexpr int B_STAGE = (BN / PAIR) * BK * 2;         // this CTA's share of B's BN rows
+  static constexpr int EPI_CHUNKS = BN / 32 / 2;               // 32-column chunks per epilogue warp
   static constexpr int TX_BYTES = PAIR * (A_STAGE + B_STAGE);  // per stage, both CTAs
   static constexpr int TILE_M = BM * PAIR;                     // rows of a (pair) tile
   static constexpr int SMEM = 1024 /*align slack*/ + STAGES * (A_STAGE + B_STAGE) + EPI_WARPS * EPI_BUF +
@@ -109,13 +111,13 @@ struct Tile {
   int split;
 };
 
-// Tiles of row block i (tile_m rows) that touch the lower triangle.
-__host__ __device__ inline int sym_row_tiles(int i, int tiles_n, int tile_m) {
-  int c = (i * tile_m + tile_m - 1) / BN + 1;
+// Tiles (bn columns wide) of row block i (tile_m rows) that touch the lower triangle.
+__host__ __device__ inline int sym_row_tiles(int i, int tiles_n, int tile_m, int bn) {
+  int c = (i * tile_m + tile_m - 1) / bn + 1;
   return c < tiles_n ? c : tiles_n;
 }
 
-template <int PAIR>
+template <int PAIR, int BN>
 __device__ inline Tile decode(const Params& p, int tile) {
   int gi = 0;
   while (gi + 1 < p.ngroups && tile >= p.g[gi + 1].tile_begin) ++gi;
@@ -132,7 +134,7 @@ __device__ inline Tile decode(const Params& p, int tile) {
   } else {
     int i = 0;
     for (;;) {
-      int cnt = sym_row_tiles(i, g.tiles_n, Cfg<PAIR>::TILE_M);
+      int cnt = sym_row_tiles(i, g.tiles_n, Cfg<PAIR, BN>::TILE_M, BN);
       if (t < cnt) break;
       t -= cnt;
       ++i;
@@ -143,7 +145,7 @@ __device__ inline Tile decode(const Params& p, int tile) {
   const int nkb = (g.K + BK - 1) / BK;
   const int kb0 = split * g.kbps;
   const int kb1 = kb0 + g.kbps < nkb ? kb0 + g.kbps : nkb;
-  return Tile{gi, b, tm * Cfg<PAIR>::TILE_M, tn * BN, kb0, kb1, split};
+  return Tile{gi, b, tm * Cfg<PAIR, BN>::TILE_M, tn * BN, kb0, kb1, split};
 }
 
 __device__ __forceinline__ float powi(float s, int p) {
@@ -180,9 +182,10 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* 
   }
 }
 
-template <typename T, int PAIR>
+template <typename T, int PAIR, int BN>
 __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant__ Params p) {
-  using Cf = Cfg<PAIR>;
+  using Cf = Cfg<PAIR, BN>;
+  constexpr int EPI_CHUNKS = Cf::EPI_CHUNKS;
   constexpr int STAGES = Cf::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -258,7 +261,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     uint32_t phase = 0;
     int issued = 0;
     for (int tile = unit; tile < p.total_tiles; tile += units) {
-      const Tile t = decode<PAIR>(p, tile);
+      const Tile t = decode<PAIR, BN>(p, tile);
       const Group& g = p.g[t.g];
       const int am0 = t.m0 + (int)rank * BM;            // this CTA's rows of A
       const int bn0 = t.n0 + (int)rank * (BN / PAIR);   // this CTA's rows of B
@@ -328,7 +331,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     constexpr int fmt = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
     bool ok = true;
     for (int tile = unit; tile < p.total_tiles && ok; tile += units) {
-      const Tile t = decode<PAIR>(p, tile);
+      const Tile t = decode<PAIR, BN>(p, tile);
       const Group& g = p.g[t.g];
       const uint32_t idesc = idesc_f16(fmt, g.a_mn, g.b_mn, BM * PAIR, BN);
       // K-major: 8-row groups 1024 B apart, one K step = 32 B inside the
@@ -394,7 +397,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = unit; tile < p.total_tiles; tile += units) {
-      const Tile t = decode<PAIR>(p, tile);
+      const Tile t = decode<PAIR, BN>(p, tile);
       const Group& g = p.g[t.g];
       const float s = g.scale ? g.scale[t.b] : 1.f;
       const float alpha = g.alpha * powi(s, g.alpha_pow);
@@ -717,13 +720,13 @@ bool make_map(CUtensorMap* m, Op t, const void* base, int64_t inner, int64_t out
 
 // Co-resident CTAs (PAIR = 1) or clusters (PAIR = 2) of the persistent
 // kernel; 0 if its attributes cannot be set.
-template <typename T, int PAIR>
+template <typename T, int PAIR, int BN>
 int max_units() {
   static bool attr_set = false;
   static int units = 0;
-  const void* fn = (const void*)tc::gemm_kernel<T, PAIR>;
+  const void* fn = (const void*)tc::gemm_kernel<T, PAIR, BN>;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Cfg<PAIR>::SMEM) != cudaSuccess)
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Cfg<PAIR, BN>::SMEM) != cudaSuccess)
       return 0;
     units = num_sms() / PAIR;
     if (PAIR == 2) {
@@ -732,7 +735,7 @@ int max_units() {
       cudaLaunchConfig_t q = {};
       q.gridDim = dim3(2 * units);
       q.blockDim = dim3(tc::THREADS);
-      q.dynamicSmemBytes = tc::Cfg<PAIR>::SMEM;
+      q.dynamicSmemBytes = tc::Cfg<PAIR, BN>::SMEM;
       cudaLaunchAttribute a[1];
       a[0].id = cudaLaunchAttributeClusterDimension;
       a[0].val.clusterDim.x = 2;
@@ -750,13 +753,13 @@ int max_units() {
   return units;
 }
 
-template <typename T, int PAIR>
+template <typename T, int PAIR, int BN>
 muon_status launch(const tc::Params& p, int total_tiles, int max_units, cudaStream_t s) {
   const int units = total_tiles < max_units ? total_tiles : max_units;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(units * PAIR);
   cfg.blockDim = dim3(tc::THREADS);
-  cfg.dynamicSmemBytes = tc::Cfg<PAIR>::SMEM;
+  cfg.dynamicSmemBytes = tc::Cfg<PAIR, BN>::SMEM;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -767,7 +770,7 @@ muon_status launch(const tc::Params& p, int total_tiles, int max_units, cudaStre
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, tc::gemm_kernel<T, PAIR>, p) == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
+  return cudaLaunchKernelEx(&cfg, tc::gemm_kernel<T, PAIR, BN>, p) == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
 }
 
 template <typename T>
@@ -792,11 +795,16 @@ constexpr int kMaxSplits = 8;
 static_assert(kMaxSplits <= tc::RED_MAX_PARTS, "the reduction holds every part in registers");
 constexpr int kMinSplitKb = 32;
 
-int sym_tiles(int64_t n, int tile_m) {
-  const int tm = (int)((n + tile_m - 1) / tile_m), tn = (int)((n + tc::BN - 1) / tc::BN);
+int sym_tiles(int64_t n, int tile_m, int bn) {
+  const int tm = (int)((n + tile_m - 1) / tile_m), tn = (int)((n + bn - 1) / bn);
   int c = 0;
-  for (int i = 0; i < tm; ++i) c += tc::sym_row_tiles(i, tn, tile_m);
+  for (int i = 0; i < tm; ++i) c += tc::sym_row_tiles(i, tn, tile_m, bn);
   return c;
+}
+
+// Tiles of one matrix of a group at tile width bn.
+int desc_tiles(const GemmDesc& d, int tile_m, int bn) {
+  return d.sym ? sym_tiles(d.M, tile_m, bn) : ((d.M + tile_m - 1) / tile_m) * ((d.N + bn - 1) / bn);
 }
 
 // Parts for a symmetric launch of `tiles` tiles over `units` CTAs (pairs)
@@ -836,7 +844,7 @@ size_t tc_split_scratch(int64_t n, int64_t K, int count) {
     // num_sms() / pair bounds the co-resident units from above, so the
     // reservation covers every launch this group takes part in
     int kbps = 0;
-    const int parts = split_parts(count * sym_tiles(n, tc::BM * pair), num_sms() / pair, nkb, &kbps);
+    const int parts = split_parts(count * sym_tiles(n, tc::BM * pair, tc::BN_WIDE), num_sms() / pair, nkb, &kbps);
     if (parts > 1) {
       const size_t b = (size_t)parts * count * n * pad_ld(n) * sizeof(float);
       if (b > best) best = b;
@@ -845,31 +853,84 @@ size_t tc_split_scratch(int64_t n, int64_t K, int count) {
   return best;
 }
 
+template <int BN>
+int units_for(Op t, int pair) {
+  if (pair == 2) return t == Op::BF16 ? max_units<__nv_bfloat16, 2, BN>() : max_units<__half, 2, BN>();
+  return t == Op::BF16 ? max_units<__nv_bfloat16, 1, BN>() : max_units<__half, 1, BN>();
+}
+
+template <int BN>
+muon_status launch_for(Op t, int pair, const tc::Params& p, int total, int units, cudaStream_t s) {
+  if (pair == 2)
+    return t == Op::BF16 ? launch<__nv_bfloat16, 2, BN>(p, total, units, s) : launch<__half, 2, BN>(p, total, units, s);
+  return t == Op::BF16 ? launch<__nv_bfloat16, 1, BN>(p, total, units, s) : launch<__half, 1, BN>(p, total, units, s);
+}
+
 muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t timeout_ns, cudaStream_t s) {
   if (ngroups < 1 || ngroups > kMaxGemmGroups || (t != Op::BF16 && t != Op::F16)) return MUON_ERR_INVALID_ARG;
   const int pair = g_pair_mode;
   const int tile_m = tc::BM * pair;
-  const int units = pair == 2 ? (t == Op::BF16 ? max_units<__nv_bfloat16, 2>() : max_units<__half, 2>())
-                              : (t == Op::BF16 ? max_units<__nv_bfloat16, 1>() : max_units<__half, 1>());
+  int units = units_for<tc::BN_WIDE>(t, pair);
   if (units <= 0) return MUON_ERR_CUDA;
-  tc::Params p;
-  memset(&p, 0, sizeof(p));
+
+  // the groups that have work, their tile counts at the wide tile width,
+  // and the split of K where a symmetric launch leaves CTAs (pairs) idle
   const GemmDesc* src[kMaxGemmGroups];
-  int base_tiles[kMaxGemmGroups];
-  int total_base = 0;
-  int ng = 0;
+  int parts[kMaxGemmGroups], kbps[kMaxGemmGroups];
+  int ng = 0, total_wide = 0;
   for (int i = 0; i < ngroups; ++i) {
     const GemmDesc& d = gd[i];
     if (d.batch <= 0 || d.M <= 0 || d.N <= 0 || d.K <= 0) continue;
     if (d.ldd % 64 || (d.beta != 0.f && d.ldc % 64)) return MUON_ERR_INVALID_ARG;
     if (d.sym && d.M != d.N) return MUON_ERR_INVALID_ARG;
-    tc::Group& g = p.g[ng];
+    src[ng++] = &d;
+    total_wide += desc_tiles(d, tile_m, tc::BN_WIDE) * d.batch;
+  }
+  if (ng == 0) return MUON_OK;
+  bool any_split = false;
+  for (int i = 0; i < ng; ++i) {
+    const GemmDesc& d = *src[i];
+    const int nkb = (d.K + tc::BK - 1) / tc::BK;
+    parts[i] = 1;
+    kbps[i] = nkb;
+    if (!d.sym || !d.part) continue;
+    int per = 0;
+    const int n = split_parts(total_wide, units, nkb, &per);
+    if (n < 2 || (size_t)n * d.batch * d.N * pad_ld(d.N) * sizeof(float) > d.part_bytes) continue;
+    parts[i] = n;
+    kbps[i] = per;
+    any_split = true;
+  }
+  // A launch that still leaves CTAs (pairs) idle and is not split takes
+  // 128-column tiles when they all fit in one wave: twice the tiles, each
+  // with half the MMAs and half the epilogue.
+  int bn = tc::BN_WIDE;
+  if (!any_split && total_wide < units) {
+    int total_narrow = 0;
+    for (int i = 0; i < ng; ++i) total_narrow += desc_tiles(*src[i], tile_m, tc::BN_NARROW) * src[i]->batch;
+    const int units_narrow = units_for<tc::BN_NARROW>(t, pair);
+    if (units_narrow <= 0) return MUON_ERR_CUDA;
+    if (total_narrow > total_wide && total_narrow <= units_narrow) {
+      bn = tc::BN_NARROW;
+      units = units_narrow;
+    }
+  }
+
+  tc::Params p;
+  memset(&p, 0, sizeof(p));
+  tc::SplitParams sp;
+  memset(&sp, 0, sizeof(sp));
+  int base_tiles[kMaxGemmGroups];
+  int red_blocks = 0;
+  for (int i = 0; i < ng; ++i) {
+    const GemmDesc& d = *src[i];
+    tc::Group& g = p.g[i];
     // A operand source: K-major [M][K], MN-major [K][M]; 128 rows per CTA.
-    // B operand source: K-major [N][K], MN-major [K][N]; 256 / pair rows per CTA.
+    // B operand source: K-major [N][K], MN-major [K][N]; bn / pair rows per CTA.
     bool ok = d.a_mn ? make_map(&g.tmA, t, d.A, d.M, d.K, d.batch, d.lda, d.strideA, 64)
                      : make_map(&g.tmA, t, d.A, d.K, d.M, d.batch, d.lda, d.strideA, tc::BM);
     ok = ok && (d.b_mn ? make_map(&g.tmB, t, d.B, d.N, d.K, d.batch, d.ldb, d.strideB, 64)
-                       : make_map(&g.tmB, t, d.B, d.K, d.N, d.batch, d.ldb, d.strideB, tc::BN / pair));
+                       : make_map(&g.tmB, t, d.B, d.K, d.N, d.batch, d.ldb, d.strideB, bn / pair));
     ok = ok && make_map(&g.tmD, t, d.D, d.N, d.M, d.batch, d.ldd, d.strideD, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
     if (!ok) return MUON_ERR_CUDA;
     g.D = d.D;
@@ -892,34 +953,15 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
     g.beta = d.beta;
     g.gamma = d.gamma;
     g.tiles_m = (d.M + tile_m - 1) / tile_m;
-    g.tiles_n = (d.N + tc::BN - 1) / tc::BN;
-    g.tiles_per_batch = d.sym ? sym_tiles(d.M, tile_m) : g.tiles_m * g.tiles_n;
-    g.splits = 1;
-    g.kbps = (d.K + tc::BK - 1) / tc::BK;
-    src[ng] = &d;
-    base_tiles[ng] = g.tiles_per_batch;
-    total_base += g.tiles_per_batch * d.batch;
-    ++ng;
-  }
-  if (ng == 0) return MUON_OK;
-
-  // split K where the launch leaves CTAs (pairs) idle and a scratch is given
-  tc::SplitParams sp;
-  memset(&sp, 0, sizeof(sp));
-  int red_blocks = 0;
-  for (int i = 0; i < ng; ++i) {
-    tc::Group& g = p.g[i];
-    const GemmDesc& d = *src[i];
-    if (!d.sym || !d.part) continue;
-    int kbps = 0;
-    const int parts = split_parts(total_base, units, g.kbps, &kbps);
+    g.tiles_n = (d.N + bn - 1) / bn;
+    base_tiles[i] = desc_tiles(d, tile_m, bn);
+    g.tiles_per_batch = base_tiles[i] * parts[i];
+    g.splits = parts[i];
+    g.kbps = kbps[i];
+    if (parts[i] < 2) continue;
     const int64_t ldp = pad_ld(d.N);
-    if (parts < 2 || (size_t)parts * d.batch * d.N * ldp * sizeof(float) > d.part_bytes) continue;
-    if (!make_map(&g.tmP, Op::F32, d.part, d.N, d.M, (int64_t)parts * d.batch, ldp, (int64_t)d.M * ldp, 32, 32))
+    if (!make_map(&g.tmP, Op::F32, d.part, d.N, d.M, (int64_t)parts[i] * d.batch, ldp, (int64_t)d.M * ldp, 32, 32))
       return MUON_ERR_CUDA;
-    g.splits = parts;
-    g.kbps = kbps;
-    g.tiles_per_batch *= parts;
     tc::SplitGroup& r = sp.g[sp.ngroups++];
     r.part = d.part;
     r.D = d.D;
@@ -932,7 +974,7 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
     r.sC = d.strideC;
     r.n = d.N;
     r.batch = d.batch;
-    r.splits = parts;
+    r.splits = parts[i];
     r.nb32 = (d.N + 31) / 32;
     r.blocks_per_batch = r.nb32 * (r.nb32 + 1) / 2;
     r.block_begin = red_blocks;
@@ -966,13 +1008,10 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
     const double mnk = (double)g.M * g.N * g.K * g.batch;
     cn.flops_dense += 2.0 * mnk;
     cn.flops_sym += g.sym ? mnk : 2.0 * mnk;
-    cn.flops_exec += 2.0 * tile_m * tc::BN * (double)g.K * base_tiles[i] * g.batch;
+    cn.flops_exec += 2.0 * tile_m * bn * (double)g.K * base_tiles[i] * g.batch;
   }
-  muon_status r;
-  if (pair == 2)
-    r = t == Op::BF16 ? launch<__nv_bfloat16, 2>(p, total, units, s) : launch<__half, 2>(p, total, units, s);
-  else
-    r = t == Op::BF16 ? launch<__nv_bfloat16, 1>(p, total, units, s) : launch<__half, 1>(p, total, units, s);
+  const muon_status r = bn == tc::BN_WIDE ? launch_for<tc::BN_WIDE>(t, pair, p, total, units, s)
+                                          : launch_for<tc::BN_NARROW>(t, pair, p, total, units, s);
   if (r != MUON_OK || sp.ngroups == 0) return r;
   return t == Op::BF16 ? launch_reduce<__nv_bfloat16>(sp, red_blocks, s) : launch_reduce<__half>(sp, red_blocks, s);
 }
