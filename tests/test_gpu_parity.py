@@ -431,3 +431,21 @@ def test_split_k_dion3_batched_step():
     assert st == mu.OK
     k = O.rows_for_fraction(1024, 1, 4)
     check_step(state, got, O.StepParams(gram=True, restart_at=3, normuon=True, k=k, select_norm="l2"), TOL16)
+
+
+@pytest.mark.parametrize("pair", [True, False])
+@pytest.mark.parametrize("gram", [False, True])
+def test_narrow_tiles_ragged(pair, gram):
+    """Launches too small to fill the GPU run on 128-column tiles (256x128
+    per CTA pair, 128x128 per CTA): ragged symmetric n (300, 200) and
+    rectangular groups, standard bf16 and Gram fp16, both kernel forms."""
+    shapes = [(300, 700), (300, 700), (700, 300), (200, 200), (130, 390)]
+    state = make_state(shapes, 9500 + 10 * pair + gram, m_std=1e-3)
+    p = mu.step_params(ns=mu.ns_params(gram=gram, restart_at=3, compute=mu.F16 if gram else mu.BF16))
+    mu.set_gemm_cta_pair(pair)
+    try:
+        got, st = run_step(state, p)
+    finally:
+        mu.set_gemm_cta_pair(True)
+    assert st == mu.OK, mu.status_str(st)
+    check_step(state, got, O.StepParams(gram=gram, restart_at=3), TOL16)
