@@ -1,47 +1,50 @@
 // Tensor-core GEMM for the Newton-Schulz chain on sm_100a.
 //
 // Persistent, warp-specialised kernel, one CTA per SM, 384 threads, in two
-// forms sharing everything but the mainloop's data movement:
-//   PAIR = 1  one CTA computes a 128x256 tile: tcgen05.mma cta_group::1,
-//             M = 128, N = 256; 4-stage ring of 48 KB (A 128x64, B 256x64).
-//   PAIR = 2  a cluster of two CTAs computes a 256x256 tile: the leader issues
-//             tcgen05.mma cta_group::2, M = 256, N = 256, reading A's 128 rows
-//             and B's 128 rows from each CTA's own shared memory; each CTA
-//             TMA-loads only its halves (32 KB per k-block instead of 48 KB
-//             of operand traffic per SM) into a 6-stage ring, and the copy
-//             completions are counted on the leader's barrier. MMA
-//             completions are signalled to both CTAs' barriers.
+// forms sharing everything but the mainloop's data movement, each with
+// BN = 256 or 128 tile columns:
+//   PAIR = 1  one CTA computes a 128xBN tile: tcgen05.mma cta_group::1,
+//             M = 128, N = BN; ring of 4 (BN 256) or 6 (BN 128) stages.
+//   PAIR = 2  a cluster of two CTAs computes a 256xBN tile: the leader issues
+//             tcgen05.mma cta_group::2, M = 256, N = BN, reading A's 128 rows
+//             and B's BN/2 rows from each CTA's own shared memory; each CTA
+//             TMA-loads only its halves into a ring of 6 (BN 256) or 8
+//             (BN 128) stages, and the copy completions are counted on the
+//             leader's barrier. MMA completions are signalled to both CTAs'
+//             barriers.
 // Roles:
 //   warps 0, 3  TMA producers (one thread each: A boxes, B boxes), 128-byte swizzle
 //   warp 1      MMA issuer (one thread of the leader), fp32 accumulators in TMEM
-//   warp 2      allocates / frees the 512 TMEM columns (two 128x256 fp32
+//   warp 2      allocates / frees the 512 TMEM columns (two 128xBN fp32
 //               accumulators: the epilogue of tile i overlaps the mainloop of
 //               tile i+1)
-//   warps 4..11 epilogue, two warps per TMEM lane quarter, each owning 128
-//               of the tile's 256 columns: C rows prefetched into registers,
-//               tcgen05.ld of 32x32 sub-tiles, fused alpha*acc + beta*C +
-//               gamma*I, one rounding to the stored type, then each 32x32
-//               block is staged in 64B-swizzled shared memory and written by
-//               a TMA bulk tensor store (clipped at the matrix edge). For
-//               symmetric outputs a second staged block holds the transpose,
-//               stored at the mirrored position; a block on the diagonal is
-//               symmetrised in shared memory and stored once.
+//   warps 4..11 epilogue, two warps per TMEM lane quarter, each owning BN/2
+//               of the tile's columns: C blocks loaded (coalesced) before the
+//               accumulator wait, 32x32 sub-tiles read from TMEM in the
+//               m16n8 fragment layout, fused alpha*acc + beta*C + gamma*I,
+//               one rounding to the stored type, then each 32x32 block is
+//               staged with stmatrix in 64B-swizzled shared memory and
+//               written by a TMA bulk tensor store (clipped at the matrix
+//               edge). For symmetric outputs stmatrix.trans stages the
+//               transpose, stored at the mirrored position; a block on the
+//               diagonal is symmetrised in shared memory and stored once.
 //
 // Symmetric outputs ("2. Symmetric GEMM Kernels" of the Dion3 page: a
 // triangular scheduler over lower tiles and a transposed-tile epilogue) are
 // scheduled over the tiles that touch the lower triangle only.
 //
-// Split K: a symmetric launch with fewer tiles than the GPU has CTAs (or
-// pairs), e.g. X X^T of a 2048-row matrix with K = 16384, may split each
-// tile's K range into `splits` contiguous parts, one work unit each. Such a
-// unit stores its raw fp32 accumulator (lower sub-tiles only) to a partial
-// buffer, and split_reduce_kernel then sums the parts in a fixed order,
-// applies the epilogue and writes the direct and mirrored copies, so the
-// result is deterministic and exactly symmetric.
+// Small launches: a launch whose 256-column tiles leave CTAs (pairs) idle
+// either splits K (symmetric X X^T with a long K: each tile's k-blocks in
+// `splits` contiguous parts, one work unit each, raw fp32 accumulators to a
+// partial buffer, then split_reduce_kernel sums the parts in a fixed order,
+// applies the epilogue and writes both triangles, so the result is
+// deterministic and exactly symmetric) or, when not split, runs on
+// 128-column tiles if they all fit in one wave.
 //
 // Every wait is bounded (mbar_wait_bounded): on expiry the kernel records
 // MUON_ERR_TIMEOUT, every role stops, in-flight copies and MMAs are drained
 // with bounded waits and TMEM is freed before the CTA exits.
+#include <atomic>
 #include <cstring>
 #include <mutex>
 #include <type_traits>
@@ -718,22 +721,37 @@ bool make_map(CUtensorMap* m, Op t, const void* base, int64_t inner, int64_t out
   return r == CUDA_SUCCESS;
 }
 
+constexpr int kMaxDevices = 64;
+
+int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) {
+    cudaGetLastError();
+    d = 0;
+  }
+  return d;
+}
+
 // Co-resident CTAs (PAIR = 1) or clusters (PAIR = 2) of the persistent
-// kernel; 0 if its attributes cannot be set.
+// kernel on the current device; 0 if its attributes cannot be set. The
+// shared-memory attribute is set, and the count taken, once per device.
 template <typename T, int PAIR, int BN>
 int max_units() {
-  static bool attr_set = false;
-  static int units = 0;
+  static std::mutex mu;
+  static int per_device[kMaxDevices];  // 0: not set up on that device yet
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lock(mu);
+  int& units = per_device[dev];
   const void* fn = (const void*)tc::gemm_kernel<T, PAIR, BN>;
-  if (!attr_set) {
+  if (units == 0) {
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Cfg<PAIR, BN>::SMEM) != cudaSuccess)
       return 0;
-    units = num_sms() / PAIR;
+    int u = num_sms() / PAIR;
     if (PAIR == 2) {
       // not every SM may have a free partner in its GPC: launch only as many
       // persistent pairs as can run at once
       cudaLaunchConfig_t q = {};
-      q.gridDim = dim3(2 * units);
+      q.gridDim = dim3(2 * u);
       q.blockDim = dim3(tc::THREADS);
       q.dynamicSmemBytes = tc::Cfg<PAIR, BN>::SMEM;
       cudaLaunchAttribute a[1];
@@ -744,11 +762,11 @@ int max_units() {
       q.attrs = a;
       q.numAttrs = 1;
       int clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&clusters, fn, &q) == cudaSuccess && clusters > 0 && clusters < units)
-        units = clusters;
+      if (cudaOccupancyMaxActiveClusters(&clusters, fn, &q) == cudaSuccess && clusters > 0 && clusters < u)
+        u = clusters;
       cudaGetLastError();
     }
-    attr_set = true;
+    units = u;
   }
   return units;
 }
@@ -826,11 +844,15 @@ int split_parts(int tiles, int units, int nkb, int* kbps) {
 }  // namespace
 
 int num_sms() {
-  static int n = 0;
+  static std::atomic<int> per_device[kMaxDevices];  // 0: not queried yet
+  const int dev = current_device();
+  int n = per_device[dev].load(std::memory_order_relaxed);
   if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = 148;  // no device here (workspace planning on a host without a GPU)
+    }
+    per_device[dev].store(n, std::memory_order_relaxed);
   }
   return n;
 }

@@ -461,29 +461,25 @@ __device__ void normuon_finalize_block(float* rscale, int64_t k, int64_t m, floa
   for (int64_t i = threadIdx.x; i < k; i += BLOCK) rscale[i] = ratio * rscale[i];
 }
 
-// cols % 4 == 0: vectors of 4, UNROLL of them in flight per thread
+// cols % 4 == 0: block (row, chunk of BLOCK * UNROLL vectors of 4), UNROLL
+// vectors in flight per thread, no index division.
 template <typename I, typename O>
-__global__ void __launch_bounds__(BLOCK) copy_out4(const I* in, int64_t ldi, O* out, int64_t rows, int64_t cols) {
-  const int64_t n4 = cols >> 2, total = rows * n4;
-  const int64_t stride = (int64_t)gridDim.x * BLOCK;
-  for (int64_t e0 = blockIdx.x * (int64_t)BLOCK + threadIdx.x; e0 < total; e0 += stride * UNROLL) {
-    float4 v[UNROLL];
+__global__ void __launch_bounds__(BLOCK) copy_out4(const I* in, int64_t ldi, O* out, int64_t cols) {
+  const int64_t r = blockIdx.x;
+  const int64_t n4 = cols >> 2;
+  const int64_t c0 = (int64_t)blockIdx.y * (BLOCK * UNROLL) + threadIdx.x;
+  const I* src = in + r * ldi;
+  O* dst = out + r * cols;
+  float4 v[UNROLL];
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const int64_t e = e0 + u * stride;
-      if (e < total) {
-        const int64_t r = e / n4, c = (e - r * n4) << 2;
-        v[u] = Src<I>::load4(in + r * ldi + c);
-      }
-    }
+  for (int u = 0; u < UNROLL; ++u) {
+    const int64_t c = c0 + u * BLOCK;
+    if (c < n4) v[u] = Src<I>::load4(src + 4 * c);
+  }
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const int64_t e = e0 + u * stride;
-      if (e < total) {
-        const int64_t r = e / n4, c = (e - r * n4) << 2;
-        Dst<O>::store4(out + r * cols + c, v[u]);
-      }
-    }
+  for (int u = 0; u < UNROLL; ++u) {
+    const int64_t c = c0 + u * BLOCK;
+    if (c < n4) Dst<O>::store4(dst + 4 * c, v[u]);
   }
 }
 
@@ -659,11 +655,14 @@ muon_status launch_copy_out(const void* in, Op it, int64_t ldi, void* out, Op ot
   if (total == 0) return MUON_OK;
   int64_t g = (total + BLOCK - 1) / BLOCK;
   if (g > 148 * 16) g = 148 * 16;
-  const bool v4 = (cols & 3) == 0;  // rows of out then start on 16-byte (f32) / 8-byte (bf16) boundaries
+  // rows of out start on 16-byte (f32) / 8-byte (bf16) boundaries when cols % 4 == 0
+  const int64_t chunks = ((cols >> 2) + BLOCK * UNROLL - 1) / (BLOCK * UNROLL);
+  const bool v4 = (cols & 3) == 0 && rows <= INT32_MAX && chunks <= 65535;
+  const dim3 g4((unsigned)rows, (unsigned)chunks);
 #define CP(I, O)                                                                                             \
   do {                                                                                                       \
-    if (v4) copy_out4<I, O><<<(int)g, BLOCK, 0, s>>>(reinterpret_cast<const I*>(in), ldi, reinterpret_cast<O*>(out), rows, cols); \
-    else copy_out<I, O><<<(int)g, BLOCK, 0, s>>>(reinterpret_cast<const I*>(in), ldi, reinterpret_cast<O*>(out), rows, cols);     \
+    if (v4) copy_out4<I, O><<<g4, BLOCK, 0, s>>>(reinterpret_cast<const I*>(in), ldi, reinterpret_cast<O*>(out), cols); \
+    else copy_out<I, O><<<(int)g, BLOCK, 0, s>>>(reinterpret_cast<const I*>(in), ldi, reinterpret_cast<O*>(out), rows, cols); \
   } while (0)
   if (it == Op::F32) { if (ot == Op::F32) CP(float, float); else CP(float, __nv_bfloat16); }
   else if (it == Op::F16) { if (ot == Op::F32) CP(__half, float); else CP(__half, __nv_bfloat16); }
