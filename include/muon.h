@@ -144,7 +144,11 @@ int64_t muon_rows_for_fraction(int64_t n, int32_t f_num, int32_t f_den);
 void muon_ns_params_default(muon_ns_params* p);
 
 /* Workspace bytes needed by ns_polar / gram_ns_polar for one rows x cols
- * matrix with parameters p (returns 0 for invalid arguments). */
+ * matrix with parameters p (returns 0 for invalid arguments). Includes the
+ * fp32 scratch that X X^T products of a short, wide matrix use to split
+ * their inner dimension across the GPU; that part depends on the SM count
+ * of the current device, so query with the device that will run the call
+ * current. */
 size_t muon_ns_workspace_size(int64_t rows, int64_t cols, const muon_ns_params* p);
 
 /* O ~= polar(X) by T quintic Newton-Schulz steps ("Standard Newton-Schulz";
@@ -212,7 +216,8 @@ muon_status select_rows_noalloc(const float* M, int64_t n, int64_t m, int64_t k,
                                 int32_t* idx_out, int32_t* dev_status, void* stream);
 
 /* Workspace bytes for muon_step over mats[0..count) with parameters p
- * (0 for invalid arguments). */
+ * (0 for invalid arguments). Like muon_ns_workspace_size, query with the
+ * device that will run the step current. */
 size_t muon_workspace_size(const muon_matrix* mats, int32_t count, const muon_params* p);
 
 /* One optimizer step over count independent matrices (host array mats):
@@ -228,8 +233,8 @@ muon_status muon_step(const muon_matrix* mats, int32_t count, const muon_params*
  * Newton-Schulz products: ns_flops counts a product with a symmetric result
  * as one triangle (the page's FLOP analysis for symmetric GEMMs),
  * ns_flops_dense counts every product as 2 m n k, ns_flops_executed is the
- * tensor-core work actually issued (whole 128x256 tiles, diagonal tiles in
- * full). Bytes are the compulsory HBM bytes of the memory-bound phases. */
+ * tensor-core work actually issued (whole tiles of 128 or 256 rows by 128
+ * or 256 columns, diagonal tiles in full). Bytes are the compulsory HBM bytes of the memory-bound phases. */
 typedef struct {
   float ms_total;
   float ms_prologue;   /* momentum, norms, selection, operand casts */
