@@ -428,14 +428,23 @@ def run_spectrum(args, rank, world, local_rank):
         X = inputs.gaussian((n, m), 1.0, 6000, 0)
     Xd = torch.from_numpy(X.astype(np.float32)).cuda().to(torch.bfloat16)
     del X
-    variants = [("gram_f16", mu.ns_params(gram=True, restart_at=3, compute=mu.F16), True),
-                ("standard_bf16", mu.ns_params(compute=mu.BF16), False),
-                ("standard_f16", mu.ns_params(compute=mu.F16), False)]
+    variants = [("gram_f16", mu.ns_params(gram=True, restart_at=3, compute=mu.F16), True, 5),
+                ("standard_bf16", mu.ns_params(compute=mu.BF16), False, 5),
+                ("standard_f16", mu.ns_params(compute=mu.F16), False, 5)]
+    if args.workload == "spectrum4096x16384":
+        # tuned per-step schedules (minimax quintics): orthogonality error
+        # against the step count, i.e. the FLOP budget
+        from newton_schulz_10_b200 import schedules
+        for T, lower in ((5, 1e-3), (10, 1e-5)):
+            co, _ = schedules.minimax_schedule(T, lower)
+            variants.append((f"standard_bf16_minimax_T{T}", mu.ns_params(T=T, coeffs=co, compute=mu.BF16), False, T))
+            variants.append((f"gram_f16_minimax_T{T}",
+                             mu.ns_params(T=T, coeffs=co, gram=True, restart_at=3, compute=mu.F16), True, T))
     stream = torch.cuda.current_stream()
     res = {}
     clocks = None
     launches = 0
-    for name, p, gram in variants:
+    for name, p, gram, T in variants:
         O, ws = mu.ns_polar(Xd, p, out_dtype=torch.bfloat16)
         for _ in range(args.warmup):
             mu.ns_polar(Xd, p, out_dtype=torch.bfloat16, ws=ws)
@@ -458,7 +467,7 @@ def run_spectrum(args, rank, world, local_rank):
             launches = mu.kernel_launch_count() - n0
         Of = O.float()
         orth = float(torch.linalg.matrix_norm(Of @ Of.T - torch.eye(n, device="cuda")).item())
-        fl = ns_flops(n, m, 5, gram)
+        fl = ns_flops(n, m, T, gram)
         res[name] = {"ms": round(ms, 3), "tflops_algorithmic": round(fl / (ms * 1e-3) / 1e12, 1),
                      "orthogonality_error_fro": round(orth, 4),
                      "status": mu.status_str(int(ws[:4].view(torch.int32).item()))}
