@@ -435,11 +435,15 @@ def run_spectrum(args, rank, world, local_rank):
         # tuned per-step schedules (minimax quintics): orthogonality error
         # against the step count, i.e. the FLOP budget
         from newton_schulz_10_b200 import schedules
-        for T, lower in ((5, 1e-3), (10, 1e-5)):
-            co, _ = schedules.minimax_schedule(T, lower)
-            variants.append((f"standard_bf16_minimax_T{T}", mu.ns_params(T=T, coeffs=co, compute=mu.BF16), False, T))
-            variants.append((f"gram_f16_minimax_T{T}",
-                             mu.ns_params(T=T, coeffs=co, gram=True, restart_at=3, compute=mu.F16), True, T))
+        # (the Gram chain, with its single restart, is kept to the short
+        # table: over ten steep steps its fp16 R drifts and overflows)
+        co5, _ = schedules.minimax_schedule(5, 1e-3)
+        co10, _ = schedules.minimax_schedule(10, 1e-5)
+        variants += [("standard_bf16_minimax_T5", mu.ns_params(T=5, coeffs=co5, compute=mu.BF16), False, 5),
+                     ("gram_f16_minimax_T5", mu.ns_params(T=5, coeffs=co5, gram=True, restart_at=3, compute=mu.F16),
+                      True, 5),
+                     ("standard_bf16_minimax_T10", mu.ns_params(T=10, coeffs=co10, compute=mu.BF16), False, 10),
+                     ("standard_f16_minimax_T10", mu.ns_params(T=10, coeffs=co10, compute=mu.F16), False, 10)]
     stream = torch.cuda.current_stream()
     res = {}
     clocks = None

@@ -20,7 +20,8 @@
  *   legacy default stream). Host-side argument errors are returned before any
  *   work is queued; nothing is launched in that case.
  * - Pointers to matrices must be 16-byte aligned (MUON_ERR_ALIGN otherwise).
- * - Errors found on the device (a non-finite norm, a device wait that ran out)
+ * - Errors found on the device (a non-finite norm, a non-finite polar output
+ *   such as an fp16 overflow, a device wait that ran out)
  *   cannot be returned synchronously: they are written, as a muon_status
  *   value, to a device int32 status word. The status word is `dev_status`
  *   where a call takes one and it is non-NULL, else the first 4 bytes of the
@@ -47,7 +48,7 @@ typedef enum {
   MUON_ERR_ALIGN = 4,        /* a matrix pointer is not 16-byte aligned       */
   MUON_ERR_WORKSPACE = 5,    /* workspace NULL or smaller than required       */
   MUON_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed             */
-  MUON_ERR_NONFINITE = 7,    /* (device) a norm or ratio was not finite       */
+  MUON_ERR_NONFINITE = 7,    /* (device) a norm, ratio or output not finite   */
   MUON_ERR_TIMEOUT = 8,      /* (device) a bounded device wait ran out        */
   MUON_ERR_UNSUPPORTED = 9   /* valid request this build cannot serve         */
 } muon_status;

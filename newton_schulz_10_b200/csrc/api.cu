@@ -190,7 +190,8 @@ muon_status polar_impl(const void* X, muon_dtype x_dtype, void* O, muon_dtype o_
   g.part = q.g.part_bytes ? at<float>(ws, q.g.part) : nullptr;
   g.part_bytes = q.g.part_bytes;
   TRY(ns_run(t, &g, 1, &pp, status, timeout_ns(), s));
-  return launch_copy_out(g.X[g.cur], t, pad_ld(cols), O, o_dtype == MUON_F32 ? Op::F32 : Op::BF16, rows, cols, s);
+  return launch_copy_out(g.X[g.cur], t, pad_ld(cols), O, o_dtype == MUON_F32 ? Op::F32 : Op::BF16, rows, cols,
+                         status, s);
 }
 
 // ---------------------------------------------------------------------------

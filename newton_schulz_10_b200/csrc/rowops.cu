@@ -74,6 +74,15 @@ template <typename T> struct DstH {
 template <> struct Dst<__nv_bfloat16> : DstH<__nv_bfloat16> {};
 template <> struct Dst<__half> : DstH<__half> {};
 
+// Non-finite output of the Newton-Schulz chain (an fp16 overflow, a NaN that
+// entered through the input): reported once per warp as MUON_ERR_NONFINITE.
+__device__ __forceinline__ bool finite4(float4 v) {
+  return isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
+}
+__device__ __forceinline__ void report_if_any(bool bad, int* status) {
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) report(status, MUON_ERR_NONFINITE);
+}
+
 // ---------------------------------------------------------------------------
 // momentum + fused reductions + cast
 // ---------------------------------------------------------------------------
@@ -261,9 +270,11 @@ __global__ void __launch_bounds__(BLOCK) update_rows(const __grid_constant__ Row
   float* W = m.W + j * m.cols;
   float* M = DECAY ? m.M + j * m.cols : nullptr;
   const float mu = L.mu;
+  bool bad = false;
   if ((m.cols & 3) == 0) {
     for (int64_t c = l; c < (m.cols >> 2); c += WG) {
       const float4 ov = Src<T>::load4(o + 4 * c);
+      bad |= !finite4(ov);
       float4 w = *reinterpret_cast<const float4*>(W + 4 * c);
       w.x = fmaf(step, ov.x, w.x); w.y = fmaf(step, ov.y, w.y); w.z = fmaf(step, ov.z, w.z); w.w = fmaf(step, ov.w, w.w);
       *reinterpret_cast<float4*>(W + 4 * c) = w;
@@ -275,10 +286,13 @@ __global__ void __launch_bounds__(BLOCK) update_rows(const __grid_constant__ Row
     }
   } else {
     for (int64_t c = l; c < m.cols; c += WG) {
-      W[c] = fmaf(step, Src<T>::load1(o + c), W[c]);
+      const float ov = Src<T>::load1(o + c);
+      bad |= !isfinite(ov);
+      W[c] = fmaf(step, ov, W[c]);
       if (DECAY) M[c] *= mu;
     }
   }
+  report_if_any(bad, L.status);
 }
 
 // ---------------------------------------------------------------------------
@@ -464,7 +478,7 @@ __device__ void normuon_finalize_block(float* rscale, int64_t k, int64_t m, floa
 // cols % 4 == 0: block (row, chunk of BLOCK * UNROLL vectors of 4), UNROLL
 // vectors in flight per thread, no index division.
 template <typename I, typename O>
-__global__ void __launch_bounds__(BLOCK) copy_out4(const I* in, int64_t ldi, O* out, int64_t cols) {
+__global__ void __launch_bounds__(BLOCK) copy_out4(const I* in, int64_t ldi, O* out, int64_t cols, int* status) {
   const int64_t r = blockIdx.x;
   const int64_t n4 = cols >> 2;
   const int64_t c0 = (int64_t)blockIdx.y * (BLOCK * UNROLL) + threadIdx.x;
@@ -476,20 +490,30 @@ __global__ void __launch_bounds__(BLOCK) copy_out4(const I* in, int64_t ldi, O* 
     const int64_t c = c0 + u * BLOCK;
     if (c < n4) v[u] = Src<I>::load4(src + 4 * c);
   }
+  bool bad = false;
 #pragma unroll
   for (int u = 0; u < UNROLL; ++u) {
     const int64_t c = c0 + u * BLOCK;
-    if (c < n4) Dst<O>::store4(dst + 4 * c, v[u]);
+    if (c < n4) {
+      bad |= !finite4(v[u]);
+      Dst<O>::store4(dst + 4 * c, v[u]);
+    }
   }
+  report_if_any(bad, status);
 }
 
 template <typename I, typename O>
-__global__ void __launch_bounds__(BLOCK) copy_out(const I* in, int64_t ldi, O* out, int64_t rows, int64_t cols) {
+__global__ void __launch_bounds__(BLOCK) copy_out(const I* in, int64_t ldi, O* out, int64_t rows, int64_t cols,
+                                                  int* status) {
   const int64_t total = rows * cols;
+  bool bad = false;
   for (int64_t e = blockIdx.x * (int64_t)BLOCK + threadIdx.x; e < total; e += (int64_t)gridDim.x * BLOCK) {
     const int64_t r = e / cols, c = e - r * cols;
-    Dst<O>::store1(out + e, Src<I>::load1(in + r * ldi + c));
+    const float x = Src<I>::load1(in + r * ldi + c);
+    bad |= !isfinite(x);
+    Dst<O>::store1(out + e, x);
   }
+  report_if_any(bad, status);
 }
 
 // ---------------------------------------------------------------------------
@@ -650,7 +674,7 @@ muon_status launch_normuon_finalize_batched(const NormuonMat* mats, int count, f
 }
 
 muon_status launch_copy_out(const void* in, Op it, int64_t ldi, void* out, Op ot, int64_t rows, int64_t cols,
-                            cudaStream_t s) {
+                            int* status, cudaStream_t s) {
   const int64_t total = rows * cols;
   if (total == 0) return MUON_OK;
   int64_t g = (total + BLOCK - 1) / BLOCK;
@@ -661,8 +685,8 @@ muon_status launch_copy_out(const void* in, Op it, int64_t ldi, void* out, Op ot
   const dim3 g4((unsigned)rows, (unsigned)chunks);
 #define CP(I, O)                                                                                             \
   do {                                                                                                       \
-    if (v4) copy_out4<I, O><<<g4, BLOCK, 0, s>>>(reinterpret_cast<const I*>(in), ldi, reinterpret_cast<O*>(out), cols); \
-    else copy_out<I, O><<<(int)g, BLOCK, 0, s>>>(reinterpret_cast<const I*>(in), ldi, reinterpret_cast<O*>(out), rows, cols); \
+    if (v4) copy_out4<I, O><<<g4, BLOCK, 0, s>>>(reinterpret_cast<const I*>(in), ldi, reinterpret_cast<O*>(out), cols, status); \
+    else copy_out<I, O><<<(int)g, BLOCK, 0, s>>>(reinterpret_cast<const I*>(in), ldi, reinterpret_cast<O*>(out), rows, cols, status); \
   } while (0)
   if (it == Op::F32) { if (ot == Op::F32) CP(float, float); else CP(float, __nv_bfloat16); }
   else if (it == Op::F16) { if (ot == Op::F32) CP(__half, float); else CP(__half, __nv_bfloat16); }

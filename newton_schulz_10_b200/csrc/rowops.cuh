@@ -87,6 +87,6 @@ muon_status launch_normuon_finalize_batched(const NormuonMat* mats, int count, f
 
 // Copy an internal (padded) matrix to a caller buffer (ld = cols).
 muon_status launch_copy_out(const void* in, Op it, int64_t ldi, void* out, Op ot, int64_t rows, int64_t cols,
-                            cudaStream_t s);
+                            int* status, cudaStream_t s);
 
 }  // namespace muon
