@@ -93,3 +93,51 @@ def test_margin_keeps_steep_steps_stable():
     for abc in coeffs:
         y = O.compose_scalar(y * 1.02, [abc])
     assert np.all(np.isfinite(y)) and y.max() < 1.2 and y.min() > 0
+
+
+# ---------------------------------------------------------------------------
+# the pins above catch plausible mistakes in the schedule code
+# ---------------------------------------------------------------------------
+
+def _one_step_remez(lo, hi, iters=60, tol=1e-13):
+    """Mistake: solve on the initial Chebyshev reference, never exchange."""
+    return S.minimax_quintic(lo, hi, iters=1)
+
+
+def _no_alternation(lo, hi, iters=60, tol=1e-13):
+    """Mistake: the levelled error term has one sign on every reference point."""
+    ref = lo + (hi - lo) * 0.5 * (1.0 - np.cos(np.pi * np.arange(4) / 3.0))
+    A = np.concatenate([S._basis(ref), np.ones((4, 1))], axis=1)
+    coef = np.linalg.solve(A, np.ones(4))[:3]
+    coef = tuple(float(v) for v in coef)
+    return coef, S._max_error(coef, lo, hi)
+
+
+def _stale_intervals(T, lower, upper=1.0, margin=0.02):
+    """Mistake: every step designed for the first interval."""
+    coeffs, iv = [], [(lower, upper)]
+    for _ in range(T):
+        abc, E = S.minimax_quintic(lower, upper)
+        coeffs.append(abc)
+        iv.append((1.0 - E, 1.0 + E))
+    return coeffs, iv
+
+
+def _fails(fn):
+    try:
+        fn()
+    except Exception:  # noqa: BLE001 - any failing pin counts
+        return True
+    return False
+
+
+@pytest.mark.parametrize("attr,mutant,pin", [
+    ("minimax_quintic", _one_step_remez, lambda: test_alternation_theorem(0.3, 1.0)),
+    ("minimax_quintic", _no_alternation, lambda: test_alternation_theorem(1e-2, 1.0)),
+    ("minimax_schedule", _stale_intervals, lambda: test_schedule_keeps_singular_values_in_its_intervals(1e-3, 5)),
+    ("CONVERGED", (15.0 / 8.0, -10.0 / 8.0, 2.0 / 8.0), test_limit_is_the_converging_quintic),
+], ids=["one-step-remez", "no-alternation", "stale-intervals", "wrong-limit"])
+def test_planted_schedule_mistake_is_caught(monkeypatch, attr, mutant, pin):
+    assert not _fails(pin)
+    monkeypatch.setattr(S, attr, mutant)
+    assert _fails(pin)
