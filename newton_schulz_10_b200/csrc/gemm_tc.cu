@@ -410,8 +410,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       // The C blocks of all its chunks (and the scale above) are loaded
       // before waiting for the accumulator, so their latency overlaps that
       // wait. Loads are coalesced: load j of a chunk covers block rows
-      // 8j..8j+7, four lanes per 64-byte row; the block is handed to
-      // lane = row through shared memory later.
+      // 8j..8j+7, four lanes per 64-byte row; the block is staged in shared
+      // memory later and read back in the fragment layout with ldmatrix.
       uint4 cv[EPI_CHUNKS][4];
       const bool part = g.splits > 1;  // store the raw fp32 partial accumulator
       const bool want_c = g.beta != 0.f && !part;  // warp-uniform
