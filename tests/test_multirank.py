@@ -63,3 +63,12 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["higher_is_better"] is False and d["cpu_baseline"]["kind"] == "oracle"
+    # the rest of the bench line's contract
+    for key in ("metric", "unit", "steps", "warmup", "ms_per_step", "scaling", "vs_baseline", "dtype", "data",
+                "config"):
+        assert key in d, key
+    assert d["config"]["workload"] == "single256x1024" and d["unit"] == "ms/step"
+    cb = d["cpu_baseline"]
+    assert cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    e2e = d["e2e"]
+    assert e2e["value"] == d["value"] and e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
