@@ -259,9 +259,11 @@ __global__ void __launch_bounds__(BLOCK) normuon_rows(const __grid_constant__ Ro
 
 template <int WG, typename T, bool DECAY>
 __global__ void __launch_bounds__(BLOCK) update_rows(const __grid_constant__ RowLaunch L) {
-  const int task = blockIdx.x * (BLOCK / WG) + threadIdx.x / WG;
   const int l = threadIdx.x % WG;
-  if (task >= L.total_tasks) return;
+  // persistent: the block walks row groups with a block-uniform stride
+  for (int task0 = blockIdx.x * (BLOCK / WG); task0 < L.total_tasks; task0 += gridDim.x * (BLOCK / WG)) {
+  const int task = task0 + threadIdx.x / WG;
+  if (task >= L.total_tasks) break;
   const RowMat& m = L.m[find_mat(L, task)];
   const int64_t i = task - m.task_begin;
   const int64_t j = m.idx ? (int64_t)m.idx[i] : i;
@@ -293,6 +295,7 @@ __global__ void __launch_bounds__(BLOCK) update_rows(const __grid_constant__ Row
     }
   }
   report_if_any(bad, L.status);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -533,6 +536,14 @@ int grid_for(const RowLaunch& L, bool block) {
   return block ? L.total_tasks : (L.total_tasks + (BLOCK / 32) - 1) / (BLOCK / 32);
 }
 
+// Persistent grid for the update, which loops over row groups: enough blocks
+// to fill every SM several times over, never more than there is work.
+int persistent_grid(const RowLaunch& L, bool block) {
+  const int g = grid_for(L, block);
+  const int cap = num_sms() * (2048 / BLOCK);
+  return g < cap ? g : cap;
+}
+
 void finish(RowLaunch& L) {
   int t = 0;
   for (int i = 0; i < L.count; ++i) {
@@ -628,7 +639,7 @@ muon_status launch_update_rows(RowLaunch& L, Op ot, cudaStream_t s) {
   finish(L);
   if (L.total_tasks == 0) return MUON_OK;
   const bool block = use_block(L);
-  const int g = grid_for(L, block);
+  const int g = persistent_grid(L, block);
   const bool decay = L.mode == 1;
 #define UP(WG, T) (decay ? update_rows<WG, T, true><<<g, BLOCK, 0, s>>>(L) : update_rows<WG, T, false><<<g, BLOCK, 0, s>>>(L))
   if (ot == Op::F32) { if (block) UP(256, float); else UP(32, float); }
