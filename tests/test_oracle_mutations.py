@@ -173,6 +173,45 @@ def _polar_u_only(X):
     return U  # mistake: U instead of U V^T
 
 
+def _step_mutant(drop_scale=False, scatter_first=False, read_first=False):
+    """The oracle's whole step with one planted mistake in its NorMuon branch."""
+    def step(W, M, G, v, p, store=None):
+        W = np.asarray(W, np.float32)
+        M = np.asarray(M, np.float32)
+        G = np.asarray(G, np.float32)
+        rows = W.shape[0]
+        v = np.zeros(rows, np.float32) if v is None else np.asarray(v, np.float32)
+        if p.k is None:
+            M_new = OM.momentum(M, G, p.mu)
+            idx = np.arange(rows)
+        else:
+            M_new = OM.momentum_accumulate(M, G)
+            idx = OM.select_rows(M_new, p.k, p.select_norm)
+        Ow = OM.orthogonalize(M_new[idx, :], p, store=store)
+        v_new = v.copy()
+        k = len(idx)
+        src = np.arange(k) if read_first else idx          # mistake: v of the first k rows
+        v_rows, scale = OM.normuon(Ow, v[src], p.beta2, p.normuon_eps)
+        v_new[np.arange(k) if scatter_first else idx] = v_rows.astype(np.float32)  # mistake: wrong rows
+        if drop_scale:
+            scale = np.ones(k)                              # mistake: W -= lr O
+        W_new = W.copy()
+        W_new[idx, :] = (W[idx, :].astype(F64) - p.lr * scale[:, None] * Ow).astype(np.float32)
+        if p.k is not None:
+            M_new = M_new.copy()
+            M_new[idx, :] = (np.float32(p.mu) * M_new[idx, :]).astype(np.float32)
+        return {"W": W_new, "M": M_new, "v": v_new, "O": Ow, "idx": idx, "scale": scale}
+    step.__name__ = ("_step_drop_scale" if drop_scale else "_step_v_scatter_first" if scatter_first
+                     else "_step_v_read_first")
+    return step
+
+
+def normuon_step_pins():
+    return [lambda: pins.test_normuon_muon_step_closed_form((8, 20)),
+            lambda: pins.test_normuon_muon_step_closed_form((20, 8)),
+            pins.test_normuon_dion3_step_closed_form]
+
+
 CASES = [
     ("ns_iterations", _ns_iter_dropped_cubic, ns_pins),
     ("ns_iterations", _ns_iter_flipped_sign, ns_pins),
@@ -192,6 +231,9 @@ CASES = [
     ("fma_f32", _fma_double_rounded, lambda: [pins.test_fma_f32_midpoint_ties]),
     ("polar_svd", _polar_u_only,
      lambda: [lambda: pins.test_polar_svd_characterisation((4, 8)), pins.test_polar_svd_2x2_hand_value]),
+    ("muon_step", _step_mutant(drop_scale=True), normuon_step_pins),
+    ("muon_step", _step_mutant(scatter_first=True), lambda: [pins.test_normuon_dion3_step_closed_form]),
+    ("muon_step", _step_mutant(read_first=True), lambda: [pins.test_normuon_dion3_step_closed_form]),
 ]
 
 

@@ -417,3 +417,82 @@ def test_dion3_updates_only_selected_rows():
     # the selected rows are the 3 largest l1 rows of M + G
     l1 = np.abs(M1.astype(np.float64)).sum(1)
     assert set(S) == set(np.argsort(-l1)[:3])
+
+
+# ---------------------------------------------------------------------------
+# Whole steps with NorMuon ("NorMuon Variant", Eq. (2), applied to the
+# orthogonalised momentum of Eq. (1) and, for Dion3, to the selected rows of
+# Algorithm 4). The expected values come from the spectral closed form of the
+# Newton-Schulz output (numpy's SVD of the momentum) and from Eq. (2) written
+# out row by row with Python floats, not from the oracle's own code path.
+# ---------------------------------------------------------------------------
+
+
+def _ns_closed_form(X, coeffs, eps=1e-7):
+    """NS_T(X) = U diag(P(sigma / (||X||_F + eps))) V^T from numpy's SVD."""
+    U, s, Vt = np.linalg.svd(np.asarray(X, np.float64), full_matrices=False)
+    sn = s / (math.sqrt(float(np.sum(s * s))) + eps)
+    return (U * O.compose_scalar(sn, coeffs)) @ Vt
+
+
+def _eq2_by_rows(Orows, v_rows, beta2, eps):
+    """Eq. (2) one row at a time: v_i <- beta2 v_i + (1 - beta2) mean_j O_ij^2,
+    d_i = 1 / (sqrt(v_i) + eps), scale_i = d_i ||O||_F / ||diag(d) O||_F."""
+    k, m = Orows.shape
+    r = [math.fsum(float(x) * float(x) for x in Orows[i]) for i in range(k)]
+    v_new = [beta2 * float(v_rows[i]) + (1.0 - beta2) * r[i] / m for i in range(k)]
+    d = [1.0 / (math.sqrt(v) + eps) for v in v_new]
+    ratio = math.sqrt(math.fsum(r)) / math.sqrt(math.fsum(d[i] * d[i] * r[i] for i in range(k)))
+    return np.array(v_new), np.array([ratio * di for di in d])
+
+
+@pytest.mark.parametrize("shape", [(8, 20), (20, 8)])
+def test_normuon_muon_step_closed_form(shape):
+    """Plain Muon with NorMuon: W_i -= lr scale_i O_i for every stored row i,
+    v updated in place, with O the closed-form Newton-Schulz output of the
+    momentum. Rows of G have unequal norms, so the scales are far from 1 and
+    a dropped scale or a mis-scattered v changes the result."""
+    rows, cols = shape
+    g = inputs.rng(41, rows)
+    W = g.standard_normal(shape).astype(np.float32)
+    G = (g.standard_normal(shape) * np.linspace(0.2, 3.0, rows)[:, None]).astype(np.float32)
+    v0 = (0.01 + 0.2 * g.random(rows)).astype(np.float32)
+    p = O.StepParams(lr=0.1, normuon=True, beta2=0.9, normuon_eps=1e-4)
+    out = O.muon_step(W, np.zeros(shape, np.float32), G, v0, p)
+    # M0 = 0: the momentum 0.95 * 0 + G is G exactly
+    assert np.array_equal(out["M"], G)
+    Ocf = _ns_closed_form(G, p.coeffs)
+    v_want, scale = _eq2_by_rows(Ocf, v0, p.beta2, p.normuon_eps)
+    assert np.ptp(scale) > 0.2 * np.mean(scale)
+    assert rel(out["v"].astype(np.float64), v_want) < 1e-6
+    assert rel(out["W"].astype(np.float64) - W, -p.lr * scale[:, None] * Ocf) < 1e-5
+
+
+def test_normuon_dion3_step_closed_form():
+    """Dion3 with NorMuon (Algorithm 4 with Eq. (2) on the selected rows):
+    rows 2, 5, 9 and 11 carry ten times the momentum, so they are the k = 4
+    rows with the largest l1 norm. Only those rows of W and v change, v by
+    Eq. (2) from its own old values, W by lr scale_i times the closed-form
+    polar approximation of M[S]; M[S] is then multiplied by mu."""
+    n, m, k = 12, 16, 4
+    g = inputs.rng(43, 0)
+    W = g.standard_normal((n, m)).astype(np.float32)
+    M = g.standard_normal((n, m)).astype(np.float32)
+    G = g.standard_normal((n, m)).astype(np.float32)
+    S = [2, 5, 9, 11]
+    M[S] *= 10.0
+    v0 = (0.01 + 0.2 * g.random(n)).astype(np.float32)
+    p = O.StepParams(lr=0.1, normuon=True, beta2=0.9, normuon_eps=1e-4, k=k)
+    out = O.muon_step(W, M, G, v0, p)
+    assert list(out["idx"]) == S
+    M1 = (M + G).astype(np.float32)
+    Ocf = _ns_closed_form(M1[S], p.coeffs)
+    v_rows, scale = _eq2_by_rows(Ocf, v0[S], p.beta2, p.normuon_eps)
+    assert np.ptp(scale) > 0.02 * np.mean(scale)
+    others = np.setdiff1d(np.arange(n), S)
+    assert np.array_equal(out["v"][others], v0[others])
+    assert rel(out["v"][S].astype(np.float64), v_rows) < 1e-6
+    assert np.array_equal(out["W"][others], W[others])
+    assert rel(out["W"][S].astype(np.float64) - W[S], -p.lr * scale[:, None] * Ocf) < 1e-5
+    assert np.array_equal(out["M"][S], (np.float32(0.95) * M1[S]).astype(np.float32))
+    assert np.array_equal(out["M"][others], M1[others])
