@@ -468,8 +468,11 @@ def test_minimax_schedule(gram, compute):
     Steeper tables (lower end 1e-3, first-step slope 8.5) make the fp16 Gram
     chain fragile: its products are computed on one triangle and mirrored,
     which keeps the rounding residue of fp16 factors that no longer commute
-    exactly, and equally valid roundings then land anywhere in 1.3-4.5%
-    (a CPU replica of the kernel's arithmetic gives the GPU's 2.9%)."""
+    exactly, and equally valid roundings then straddle the 2e-2 bound
+    (tests/test_gram_fp16_replica.py: a CPU replica of the library's storage
+    points and one-triangle products gives 3.0% for the library's choice,
+    where the GPU gave 2.9%, and 1.3% for products computed in full; every
+    variant stays below 1% with the table from 1e-2)."""
     from newton_schulz_10_b200 import schedules
     X, _ = inputs.spectrum_matrix(256, 1024, -2.0, seed=9600)
     X32 = X.astype(np.float32)
