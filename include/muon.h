@@ -102,7 +102,9 @@ typedef struct {
  *                1: Dion3 (Algorithm 4): M <- M + G, select
  *                k = ceil(frac_num/frac_den * rows) rows by select_norm,
  *                orthogonalise M[S,:], update W[S,:], then M[S,:] <- mu M[S,:]
- *   dev_status   optional device int32 for deferred device errors (see top) */
+ *   dev_status   optional device int32 for deferred device errors (see top);
+ *                the library does not clear it: the caller sets it to
+ *                MUON_OK before the steps it wants to check */
 typedef struct {
   float mu;
   float lr;
@@ -209,10 +211,19 @@ muon_status select_rows(const float* M, int64_t n, int64_t m, int64_t k, muon_no
  * every GPU that loads the library until the process exits. n is limited to
  * 65536 rows (MUON_ERR_SHAPE beyond). The first call on each device looks up
  * the array's device address (cudaGetSymbolAddress) with that device
- * current; make that first call before any stream capture. All calls share
- * the one array: calls whose work overlaps on the GPU (different streams, or
- * different host threads, without ordering between them) race and give
- * wrong indices; calls ordered on one stream are safe. Allocates nothing. */
+ * current; make that first call before any stream capture. The address is
+ * kept for the life of the process, so do not use the library across a
+ * cudaDeviceReset; devices with index 64 or above are rejected
+ * (MUON_ERR_INVALID_ARG). All calls share the one array: calls whose work
+ * overlaps on the GPU (different streams, or different host threads, without
+ * ordering between them) race and give wrong indices; calls ordered on one
+ * stream are safe. Allocates nothing.
+ *
+ * dev_status, as for muon_step, is the caller's: the library never clears it,
+ * so the caller sets it to MUON_OK before the calls it wants to check (an
+ * error left from an earlier call stays, the first error written wins). With
+ * dev_status NULL, device-side errors (a non-finite row key) are not
+ * reported. */
 muon_status select_rows_noalloc(const float* M, int64_t n, int64_t m, int64_t k, muon_norm norm,
                                 int32_t* idx_out, int32_t* dev_status, void* stream);
 

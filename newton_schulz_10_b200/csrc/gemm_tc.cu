@@ -42,8 +42,10 @@
 // 128-column tiles if they all fit in one wave.
 //
 // Every wait is bounded (mbar_wait_bounded): on expiry the kernel records
-// MUON_ERR_TIMEOUT, every role stops, in-flight copies and MMAs are drained
-// with bounded waits and TMEM is freed before the CTA exits.
+// MUON_ERR_TIMEOUT, every role stops (in both CTAs of a pair), in-flight
+// copies and MMAs are drained with bounded waits (for a pair, by counting
+// what each producer issued: settle_pair_copies) and TMEM is freed before the
+// CTA exits.
 #include <atomic>
 #include <cstring>
 #include <mutex>
@@ -79,7 +81,7 @@ struct Cfg {
   static constexpr int TX_BYTES = PAIR * (A_STAGE + B_STAGE);  // per stage, both CTAs
   static constexpr int TILE_M = BM * PAIR;                     // rows of a (pair) tile
   static constexpr int SMEM = 1024 /*align slack*/ + STAGES * (A_STAGE + B_STAGE) + EPI_WARPS * EPI_BUF +
-                              (2 * STAGES + 5) * 8 + 16;
+                              (2 * STAGES + 5) * 8 + 32;
   static_assert(SMEM <= 232448, "exceeds the opt-in shared memory of one sm_100 CTA");
 };
 
@@ -185,6 +187,40 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* 
   }
 }
 
+// CTA-pair early exit: wait until every operand copy that either CTA issued
+// has landed, so that no copy writes into shared memory (or signals a
+// barrier) after the pair has left. The copies of both CTAs complete on the
+// leader's full[] barriers; `cnt` holds how many k-blocks each producer
+// issued (leader A, leader B, follower A, follower B). A producer issues
+// k-block j only after the MMAs consumed k-block j - STAGES, which needed
+// every producer's copies of it, so all k-blocks before max(cnt) - STAGES
+// have landed and each of the last STAGES k-blocks occupies its own stage.
+// For those, the barrier is settled for the copies that were never issued
+// (the missing transaction bytes, or the leader's arrival with the bytes that
+// were issued), then waited on with the drain bound.
+template <int PAIR, int BN>
+__device__ void settle_pair_copies(uint64_t* full, const volatile int* cnt, int* status) {
+  using Cf = Cfg<PAIR, BN>;
+  constexpr int STAGES = Cf::STAGES;
+  const int c[4] = {cnt[0], cnt[1], cnt[2], cnt[3]};
+  const uint32_t bytes[4] = {Cf::A_STAGE, Cf::B_STAGE, Cf::A_STAGE, Cf::B_STAGE};
+  int hi = 0;
+  for (int x = 0; x < 4; ++x) hi = c[x] > hi ? c[x] : hi;
+  for (int j = hi > STAGES ? hi - STAGES : 0; j < hi; ++j) {
+    uint32_t issued = 0;
+    for (int x = 0; x < 4; ++x)
+      if (j < c[x]) issued += bytes[x];
+    uint64_t* bar = &full[j % STAGES];
+    if (j < c[0]) {
+      // the leader's A producer arrived, expecting both CTAs' bytes
+      if (issued < (uint32_t)Cf::TX_BYTES) mbar_complete_tx(bar, Cf::TX_BYTES - issued);
+    } else {
+      mbar_arrive_expect_tx(bar, issued);
+    }
+    drain_wait(bar, (uint32_t)((j / STAGES) & 1), status);
+  }
+}
+
 template <typename T, int PAIR, int BN>
 __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant__ Params p) {
   using Cf = Cfg<PAIR, BN>;
@@ -203,11 +239,17 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* issued_cnt = reinterpret_cast<volatile int*>(tmem_slot + 2);  // pair: k-blocks per producer
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = PAIR == 2 ? cluster_rank() : 0;  // 0 = leader
   const int unit = PAIR == 2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int units = PAIR == 2 ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  // A role that stops early raises the other CTA's abort flag too, so that
+  // the pair stops together.
+  auto raise_peer = [&]() {
+    if (PAIR == 2) st_cluster_u32(mapa_shared(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u), 1u);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -220,6 +262,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
+    for (int i = 0; i < 4; ++i) issued_cnt[i] = 0;
     fence_mbar_init();
   }
   if (warp == 2) {
@@ -271,6 +314,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       bool ok = true;
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
         if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, budget, p.status)) {
+          raise_peer();
           ok = false;
           break;
         }
@@ -315,12 +359,13 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         }
         drain_wait(&full[stage], phase, p.status);  // the most recent use of `stage`
       }
-    } else if (*abort_flag) {
-      // The pair's copies complete on the leader's barriers, which this CTA
-      // cannot poll; on an early exit give in-flight copies time to land.
-      const uint64_t t0 = globaltimer_ns();
-      while (globaltimer_ns() - t0 < 200000ull) {
-      }
+    } else {
+      // The pair's copies complete on the leader's barriers: publish this
+      // producer's k-block count in the leader's table; on an early exit the
+      // leader settles and drains those barriers after the final cluster
+      // barrier (settle_pair_copies).
+      const uint32_t slot = smem_u32(const_cast<int*>(issued_cnt + 2 * rank + (issues_a ? 0 : 1)));
+      st_cluster_u32(mapa_shared(slot, 0), (uint32_t)issued);
     }
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ------------------------------------------------------------------
@@ -345,11 +390,15 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       // descriptor fields other than the start address, fixed for the tile;
       // start addresses (>> 4) stay below 2^14 inside the 228 KB window
       const uint64_t a_hi = smem_desc_sw128(0, a_lbo, 1024), b_hi = smem_desc_sw128(0, b_lbo, 1024);
-      if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, budget, p.status)) break;
+      if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1, abort_flag, budget, p.status)) {
+        raise_peer();
+        break;
+      }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * BN;
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
         if (!mbar_wait_bounded(&full[stage], phase, abort_flag, budget, p.status)) {
+          raise_peer();
           ok = false;
           break;
         }
@@ -432,7 +481,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       // every lane waits; the result is made warp-uniform so the warp-wide
       // tcgen05.ld below never runs with part of the warp gone
       const bool ok = mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, budget, p.status);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) raise_peer();
+        break;
+      }
       tc_fence_after();
 #pragma unroll
       for (int ch = 0; ch < EPI_CHUNKS; ++ch) {
@@ -568,6 +620,14 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
   __syncwarp();
   if (PAIR == 2) cluster_sync(); else __syncthreads();  // no CTA leaves while its pair still signals it
   tc_fence_after();
+  if (PAIR == 2) {
+    // every producer has published its count and every early stop has
+    // reached both abort flags; the follower stays resident (its shared
+    // memory receives its own copies) until the leader's drain ends
+    if (rank == 0 && threadIdx.x == 0 && *abort_flag) settle_pair_copies<PAIR, BN>(full, issued_cnt, p.status);
+    __syncwarp();
+    cluster_sync();
+  }
   if (warp == 2) {
     if (PAIR == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
     else tmem_dealloc(tmem_base, TMEM_COLS);

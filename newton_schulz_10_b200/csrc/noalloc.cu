@@ -26,13 +26,21 @@ static __device__ __align__(256) unsigned char g_select_scratch[kScratchBytes];
 constexpr int kMaxDevices = 64;
 
 // Device address of g_select_scratch on the current device, looked up once
-// per device (the symbol's host-side name is not a device address).
+// per device (the symbol's host-side name is not a device address). The
+// cached address belongs to the device's current context: after
+// cudaDeviceReset it would be stale, so the library is not to be used across
+// a device reset.
 void* scratch_for_current_device(muon_status* err) {
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
     *err = MUON_ERR_CUDA;
+    return nullptr;
+  }
+  if (dev < 0 || dev >= kMaxDevices) {  // beyond the per-device address table
+    *err = MUON_ERR_INVALID_ARG;
     return nullptr;
   }
   std::lock_guard<std::mutex> lock(mu);

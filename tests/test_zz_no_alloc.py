@@ -41,3 +41,25 @@ def test_noalloc_matches_select_rows_two_calls(cuda):
         torch.cuda.synchronize()
         assert int(status.item()) == mu.OK
         assert torch.equal(got, want), call
+
+
+@pytest.mark.gpu
+def test_noalloc_largest_size_bit_exact(cuda):
+    """n = 65536, the most rows the fixed scratch holds: its per-row sums and
+    keys then fill the array end to end. Two calls in a row (l1, then l2)
+    match select_rows bit for bit."""
+    import torch
+
+    n, m, k = 65536, 8, 16384
+    g = inputs.rng(905, 0)
+    M = g.standard_normal((n, m)).astype(np.float32)
+    M[n - 1] = M[0]      # an exact tie at the far end of the scratch
+    M[n // 2] = -M[7]
+    Md = torch.from_numpy(M).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for norm in (mu.NORM_L1, mu.NORM_L2):
+        want = mu.select_rows(Md, k, norm)
+        got = mu.select_rows_noalloc(Md, k, norm, dev_status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == mu.OK
+        assert torch.equal(got, want), norm
