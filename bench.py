@@ -1,12 +1,13 @@
 """Benchmark of the Muon optimizer step on B200 (one JSON line on rank 0).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gpt124m|...] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama7b|...] [--impl ours|reference]
 
-Default workload: the GPT-124M-shaped layer set (12 layers x {4 x 768x768,
-768x3072, 3072x768}), fp32 W/M/G, Newton-Schulz in bf16 with T = 5, one
-batched step per iteration. Under torchrun every rank runs its own replica of
-the step (the path has no cross-matrix exchange); the reported time is the
-max over ranks.
+Default workload: the Llama-7B-shaped layer set (32 layers x {4 x 4096x4096,
+4096x14336, 14336x4096}; 71 GB of fp32 W, M, G resident in HBM), Newton-Schulz
+in bf16 with T = 5, one batched step per iteration, NorMuon off for `value`
+and timed on as well under `normuon_on`. Under torchrun every rank runs its
+own replica of the step (the path has no cross-matrix exchange); the
+reported time is the max over ranks.
 
 --impl reference times the fp64 CPU oracle (the only other arm) on a bounded
 sample of the same workload, scaled to the whole step.
@@ -46,6 +47,9 @@ WORKLOADS = {
                              compute="f16", gram=True, normuon=True, dion3=(1, 4)),
     "llama7b": dict(desc="Llama-7B layer set: 32 x (4 x 4096x4096, 4096x14336, 14336x4096), bf16 NS T=5",
                     compute="bf16", gram=False, normuon=False, dion3=None),
+    "llama7b_layer": dict(desc="one layer of the Llama-7B set: 4 x 4096x4096, 4096x14336, 14336x4096, bf16 NS T=5 "
+                               "(profiling case: per-launch traffic x 32 = the full set's)",
+                          compute="bf16", gram=False, normuon=False, dion3=None),
     "llama_mlp_4096x14336": dict(desc="one Llama-7B MLP matrix 4096x14336, bf16 NS T=5 (profiling case)",
                                  compute="bf16", gram=False, normuon=False, dion3=None),
     "llama7b_normuon": dict(desc="Llama-7B layer set, bf16 NS T=5, NorMuon on",
@@ -83,6 +87,8 @@ def specs_for(name: str):
         return [inputs.MatrixSpec(8192, 28672, 4000, "x")]
     if name == "llama_mlp_4096x14336":
         return [inputs.llama7b_layer_set()[4]]
+    if name == "llama7b_layer":
+        return inputs.llama7b_layer_set(layers=1)
     if name.startswith("llama7b"):
         return inputs.llama7b_layer_set()
     raise ValueError(name)
@@ -203,26 +209,38 @@ def max_over_ranks(value: float, world: int) -> float:
     return float(t.item())
 
 
-def gemm_traffic(workload: str):
-    """Mean DRAM bytes per GEMM launch from the committed ncu summary of this
-    workload, if the kernel sources are unchanged since it was taken."""
+def source_hash(files) -> str:
+    """First 16 hex digits of the SHA-256 of the named csrc/ files, in order."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", f"gemm_kernel_{workload}.md")
-    if not os.path.exists(path):
-        return None, None
-    want = traffic = None
-    for line in open(path):
-        if line.startswith("source-sha256:"):
-            want = line.split(":", 1)[1].strip()
-        elif line.startswith("dram-bytes-per-launch:"):
-            traffic = float(line.split(":", 1)[1])
     h = hashlib.sha256()
-    for f in ("gemm_tc.cu", "common.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, "newton_schulz_10_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
-    if want is None or traffic is None or h.hexdigest()[:16] != want:
-        return None, None
-    return traffic, os.path.relpath(path, ROOT)
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, workload: str):
+    """DRAM read + write bytes of `kernel` on `workload` from the JSON
+    sidecars of the committed ncu summaries (profiles/*.json), reported only
+    while the kernel's sources hash to the value recorded with the capture.
+    `per` says what the bytes cover ("launch" or "step"). A capture taken on
+    a smaller case of the same kernel lists, under applies_to, the workloads
+    it scales to and the factor (units one launch or step processes, relative
+    to the capture). Returns (bytes, per, source) or (None, None, why)."""
+    import glob
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.json"))):
+        with open(path) as f:
+            d = json.load(f)
+        if d.get("kernel") != kernel:
+            continue
+        factor = d.get("applies_to", {}).get(workload)
+        if factor is None:
+            continue
+        rel = os.path.relpath(path, ROOT)
+        if source_hash(d["sources"]) != d["source_sha256_16"]:
+            return None, None, f"{rel}: kernel sources changed since the capture"
+        return d["dram_bytes"] * factor, d["per"], rel
+    return None, None, "no capture of this kernel for this workload"
 
 
 def measured_peaks():
@@ -234,64 +252,148 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def use_graph(args, big: bool) -> bool:
+    """CUDA-graph replay for the small layer sets (launch-bound), eager
+    launches with per-step phase events for the large ones."""
+    return bool(args.graph) if args.graph >= 0 else not big
+
+
+def config_for(args, specs=None) -> dict:
+    """The bench line's config: identical for our arm and the reference arm."""
+    cfg = WORKLOADS[args.workload]
+    specs = specs if specs is not None else specs_for(args.workload)
+    elems = sum(s.rows * s.cols for s in specs)
+    if args.workload in ("spectrum4096x16384", "moe_alpha8_2048x16384"):
+        s0 = specs[0]
+        return {"workload": args.workload, "description": cfg["desc"], "step": "one gram_ns_polar call",
+                "l2": f"bf16 input {2 * elems / 2**20:.0f} MiB plus working set, larger than L2",
+                "parallelism": "replicas" if args.gpus > 1 else "single GPU", "rows": s0.rows, "cols": s0.cols}
+    big = elems > 1_000_000_000
+    return {"workload": args.workload, "description": cfg["desc"], "matrices": len(specs), "elements": elems,
+            "state_bytes": 12 * elems, "l2": "inputs larger than L2 (fp32 W, M, G resident in HBM)",
+            "execution": "cuda_graph" if use_graph(args, big) else "eager, phase events per step",
+            "parallelism": "replicas" if args.gpus > 1 else "single GPU"}
+
+
 def end_to_end(args, state, step, stream, elems, big, world):
     """The step as a training loop drives it, through the public API with
-    host buffers: every step's gradients are copied from pinned host memory
+    host buffers. Every step's gradients are copied from pinned host memory
     to the device (on a copy stream, into one of two device buffers, so the
-    upload of step k+1 overlaps step k), the step runs, and its result, the
-    4-byte device status word, is read back to pinned host memory. W, M and v
+    upload of step k+1 overlaps step k); the step runs; its result, the
+    updated weights W and the 4-byte device status word, is read back to
+    pinned host memory. The read-back goes through a device snapshot of W
+    (a device-to-device copy right after the step) on a second copy stream,
+    so it overlaps the next step; the next snapshot waits for it. M and v
     stay resident, as optimizer state does in training."""
     import torch
     import torch.distributed as dist
 
     from newton_schulz_10_b200 import muon as mu
 
+    h2d = 4 * elems
+    d2h = 4 * elems + 4
     try:
         import psutil
         avail = psutil.virtual_memory().available
     except ImportError:
         avail = 1 << 62
-    if 4 * elems > 0.5 * avail:
-        return {"value": None, "unit": "ms/step", "h2d_bytes_per_step": 4 * elems, "d2h_bytes_per_step": 4,
-                "reason": f"pinned host gradients need {4 * elems / 1e9:.1f} GB, {avail / 1e9:.1f} GB available"}
+    free_dev, _ = torch.cuda.mem_get_info()
+    if 8 * elems > 0.5 * avail or 8 * elems > 0.9 * free_dev:
+        return {"value": None, "unit": "ms/step", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "reason": f"needs {8 * elems / 1e9:.1f} GB pinned host and device memory "
+                          f"({avail / 1e9:.1f} GB host available, {free_dev / 1e9:.1f} GB device free)"}
     hostG = [torch.empty_like(G, device="cpu").pin_memory() for (_, _, G, _) in state]
     for hg, (_, _, G, _) in zip(hostG, state):
         hg.copy_(G)
+    hostW = [torch.empty_like(W, device="cpu").pin_memory() for (W, _, _, _) in state]
+    snapW = [torch.empty_like(W) for (W, _, _, _) in state]
     # second device gradient buffer and a step bound to it (same workspace)
     G2 = [torch.empty_like(G) for (_, _, G, _) in state]
     steps = [step, mu.Step([(W, M, g2, v) for (W, M, _, v), g2 in zip(state, G2)], step.params, ws=step.ws)]
     gsets = [[G for (_, _, G, _) in state], G2]
     status_host = torch.zeros(1, dtype=torch.int32).pin_memory()
-    copy_stream = torch.cuda.Stream()
+    up_stream, down_stream = torch.cuda.Stream(), torch.cuda.Stream()
     copied = [torch.cuda.Event(), torch.cuda.Event()]
     done = [torch.cuda.Event(), torch.cuda.Event()]
+    snapped, read = torch.cuda.Event(), torch.cuda.Event()
     e2e_steps = max(2, min(args.steps, 50 if not big else 4))
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(stream)
-    copy_stream.wait_event(f0)
+    up_stream.wait_event(f0)
+    down_stream.wait_event(f0)
+    read.record(down_stream)
     for k in range(e2e_steps):
         buf = k % 2
-        with torch.cuda.stream(copy_stream):
+        with torch.cuda.stream(up_stream):
             if k >= 2:
-                copy_stream.wait_event(done[buf])  # step k-2 has finished reading this buffer
+                up_stream.wait_event(done[buf])  # step k-2 has finished reading this buffer
             for hg, g in zip(hostG, gsets[buf]):
                 g.copy_(hg, non_blocking=True)
-            copied[buf].record(copy_stream)
+            copied[buf].record(up_stream)
         stream.wait_event(copied[buf])
         steps[buf](stream)
         done[buf].record(stream)
+        stream.wait_event(read)  # the previous read-back has left the snapshot
         with torch.cuda.stream(stream):
+            for w, sw in zip(state, snapW):
+                sw.copy_(w[0], non_blocking=True)
             status_host.copy_(steps[buf].ws[:4].view(torch.int32), non_blocking=True)
+        snapped.record(stream)
+        with torch.cuda.stream(down_stream):
+            down_stream.wait_event(snapped)
+            for hw, sw in zip(hostW, snapW):
+                hw.copy_(sw, non_blocking=True)
+            read.record(down_stream)
+    stream.wait_event(read)
     f1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1) / e2e_steps, world)
-    return {"value": round(e2e_ms, 3), "unit": "ms/step", "h2d_bytes_per_step": 4 * elems, "d2h_bytes_per_step": 4,
-            "what": "G pinned host -> device on a copy stream (double-buffered, overlapping the previous step), "
-                    "step, 4-byte status word -> pinned host",
-            "steps": e2e_steps, "status": mu.status_str(int(status_host.item()))}
+    out = {"value": round(e2e_ms, 3), "unit": "ms/step", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "what": "G pinned host -> device (copy stream, double-buffered, overlapping the previous step), step, "
+                   "W snapshot on the device, W and the 4-byte status word -> pinned host (second copy stream, "
+                   "overlapping the next step)",
+           "steps": e2e_steps, "status": mu.status_str(int(status_host.item()))}
+    del hostG, hostW, snapW, G2
+    return out
+
+
+def phase_means(evs):
+    """Mean milliseconds of each phase over the timed steps' event sets."""
+    names = ("ms_prologue", "ms_ns", "ms_normuon", "ms_update")
+    sums = [0.0] * 4
+    for ev in evs:
+        for i in range(4):
+            sums[i] += ev[i].elapsed_time(ev[i + 1])
+    out = {n: s / len(evs) for n, s in zip(names, sums)}
+    out["ms_total"] = sum(out[n] for n in names)
+    return out
+
+
+def timed_eager(step, stream, steps, torch):
+    """`steps` eager steps, each recording its own phase events; returns the
+    event sets and the bracketing events."""
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for ev in evs:
+        step.timed(ev, stream)
+    e1.record(stream)
+    return evs, e0, e1
+
+
+def roofline_for(ns_flops_step, gemm_launches, ms_ns, peak, peak_src, workload, flops_exec):
+    achieved = ns_flops_step / (ms_ns * 1e-3) / 1e12
+    traffic, per, src = measured_traffic("gemm_kernel", workload)
+    return {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 NS chain)", "achieved": round(achieved, 1),
+            "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+            "traffic": traffic, "traffic_unit": "bytes per GEMM launch (DRAM read + write, ncu)",
+            "traffic_source": src, "flops_per_launch_algorithmic": ns_flops_step / max(gemm_launches, 1),
+            "peak_source": peak_src, "flops_per_step_algorithmic": ns_flops_step,
+            "flops_per_step_executed": flops_exec, "gemm_launches_per_step": gemm_launches,
+            "achieved_executed": round(flops_exec / (ms_ns * 1e-3) / 1e12, 1)}
 
 
 # ---------------------------------------------------------------------------
@@ -308,7 +410,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     cfg = WORKLOADS[args.workload]
     specs = specs_for(args.workload)
-    big = sum(s.rows * s.cols for s in specs) > 1_000_000_000
+    elems = sum(s.rows * s.cols for s in specs)
+    big = elems > 1_000_000_000
     state = []
     for s in specs:
         W, M, G = device_state(s, args.workload, torch, gen_on_device=big)
@@ -317,95 +420,126 @@ def run_ours(args, rank, world, local_rank):
     p = step_params(mu, cfg)
     step = mu.Step([tuple(x) for x in state], p)
     stream = torch.cuda.current_stream()
-    elems = sum(s.rows * s.cols for s in specs)
+    graph_mode = use_graph(args, big)
 
     for _ in range(args.warmup):
         step(stream)
     torch.cuda.synchronize()
     status = step.device_status()
-    run = step
+    prof = step.profiled(stream)  # FLOP and launch accounting of one step (and one more warm-up)
     graph = None
-    if args.graph:
+    if graph_mode:
         # capture one whole step (all its launches) in a CUDA graph, replay it
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             step(torch.cuda.current_stream())
-        run = lambda s=None: graph.replay()  # noqa: E731
         for _ in range(2):
-            run()
+            graph.replay()
         torch.cuda.synchronize()
 
-    # --- device-resident timing -------------------------------------------
+    # --- timed region (device-resident inputs) ------------------------------
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     n0 = mu.kernel_launch_count()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = None
     with ClockSampler(local_rank) as clk:
         t0 = time.time()
-        e0.record(stream)
-        for _ in range(args.steps):
-            run(stream)
-        e1.record(stream)
+        if graph is not None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(stream)
+        else:
+            evs, e0, e1 = timed_eager(step, stream, args.steps, torch)
         torch.cuda.synchronize()
         t1 = time.time()
     launches = mu.kernel_launch_count() - n0
     if graph is not None:  # replays queue no launches from the host: count the captured ones
-        launches = args.steps * step.profiled(stream).kernel_launches
+        launches = args.steps * prof.kernel_launches
     if world > 1:
         dist.barrier()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
     clocks = clk.summary(t0, t1)
+    status = step.device_status()
 
-    # --- per-phase profile (separate, untimed run) --------------------------
-    prof = step.profiled(stream)
+    # --- phases: from the timed steps' own events (eager), else from a
+    # profiled eager step of the same run (graph replays cannot be bracketed)
+    if evs is not None:
+        ph = phase_means(evs)
+        ph = {k: max_over_ranks(v, world) for k, v in ph.items()}
+        phase_src = "CUDA events of the timed steps (muon_step_events), mean over steps, max over ranks"
+    else:
+        ph = {k: getattr(prof, k) for k in ("ms_total", "ms_prologue", "ms_ns", "ms_normuon", "ms_update")}
+        phase_src = "CUDA events of a profiled eager step in the same run (the timed region replays a graph)"
+
+    peaks, peak_kind = measured_peaks()
+    long_step = ms > 100.0
+    tensor_peak = peaks["bf16_tflops_sustained" if long_step else "bf16_tflops"]
+    peak_src = f"{peak_kind} {'sustained' if long_step else 'burst'} bf16 (MEASURED_PEAKS.json)"
+    roof = None
+    if cfg["compute"] != "f32":
+        roof = roofline_for(prof.ns_flops, prof.gemm_launches, ph["ms_ns"], tensor_peak, peak_src, args.workload,
+                            prof.ns_flops_executed)
+        roof["time_source"] = phase_src
+    hbm = peaks["hbm_gbs"]
+    phases = {k: round(v, 4) for k, v in ph.items()}
+    phases["source"] = phase_src
+    phases["prologue_bytes_algorithmic"] = prof.bytes_prologue
+    phases["update_bytes_algorithmic"] = prof.bytes_update
+    phases["prologue_gbs"] = round(prof.bytes_prologue / (ph["ms_prologue"] * 1e-3) / 1e9, 1) if ph["ms_prologue"] else None
+    upd_ms = ph["ms_update"] + ph["ms_normuon"]
+    phases["update_gbs"] = round(prof.bytes_update / (upd_ms * 1e-3) / 1e9, 1) if upd_ms else None
+    phases["hbm_peak_gbs"] = hbm
+    for name, kern in (("prologue", "momentum_rows"), ("update", "update_rows")):
+        tr, per, src = measured_traffic(kern, args.workload)
+        phases[f"{name}_traffic"] = tr
+        phases[f"{name}_traffic_source"] = src
+    phases["kernel_launches_per_step"] = prof.kernel_launches
+
+    # --- NorMuon on (Llama-7B set): the same step with Eq. (2) -------------
+    normuon_on = None
+    if args.workload == "llama7b" and not args.no_normuon:
+        pn = step_params(mu, {**cfg, "normuon": True})
+        need = mu.workspace_size([tuple(x) for x in state], pn)
+        stepn = mu.Step([tuple(x) for x in state], pn, ws=step.ws if step.ws.numel() >= need else None)
+        for _ in range(2):
+            stepn(stream)
+        torch.cuda.synchronize()
+        kn = max(3, min(args.steps, 10))
+        profn = stepn.profiled(stream)
+        if world > 1:
+            dist.barrier()
+        evn, n0e, n1e = timed_eager(stepn, stream, kn, torch)
+        torch.cuda.synchronize()
+        msn = max_over_ranks(n0e.elapsed_time(n1e) / kn, world)
+        phn = {k: max_over_ranks(v, world) for k, v in phase_means(evn).items()}
+        rn = roofline_for(profn.ns_flops, profn.gemm_launches, phn["ms_ns"], tensor_peak, peak_src, args.workload,
+                          profn.ns_flops_executed)
+        normuon_on = {"ms_per_step": round(msn, 4), "steps": kn, "phases": {k: round(v, 4) for k, v in phn.items()},
+                      "ns_achieved_tflops": rn["achieved"], "ns_frac": rn["frac"], "peak": tensor_peak,
+                      "device_status": mu.status_str(stepn.device_status())}
+        del stepn
 
     # --- end to end through host buffers ------------------------------------
     if args.no_e2e:
         e2e = None
     else:
         e2e = end_to_end(args, state, step, stream, elems, big, world)
-    peaks, peak_kind = measured_peaks()
-    long_step = ms > 100.0
-    tensor_peak = peaks["bf16_tflops_sustained" if long_step else "bf16_tflops"]
-    if cfg["compute"] == "f32":
-        roof = None
-    else:
-        achieved = prof.ns_flops / (prof.ms_ns * 1e-3) / 1e12
-        traffic, traffic_src = gemm_traffic(args.workload)
-        roof = {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 NS chain)", "achieved": round(achieved, 1),
-                "peak": tensor_peak, "unit": "TFLOP/s", "frac": round(achieved / tensor_peak, 4),
-                "traffic": traffic, "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
-                "traffic_source": traffic_src,
-                "flops_per_launch_algorithmic": prof.ns_flops / max(prof.gemm_launches, 1),
-                "peak_source": f"{peak_kind} {'sustained' if long_step else 'burst'} bf16",
-                "flops_per_step_algorithmic": prof.ns_flops, "flops_per_step_executed": prof.ns_flops_executed,
-                "gemm_launches_per_step": prof.gemm_launches,
-                "achieved_executed": round(prof.ns_flops_executed / (prof.ms_ns * 1e-3) / 1e12, 1)}
-    hbm = peaks["hbm_gbs"]
-    phases = {k: round(getattr(prof, k), 4) for k in ("ms_total", "ms_prologue", "ms_ns", "ms_normuon", "ms_update")}
-    phases["prologue_gbs"] = round(prof.bytes_prologue / (prof.ms_prologue * 1e-3) / 1e9, 1) if prof.ms_prologue else None
-    upd_ms = prof.ms_update + prof.ms_normuon
-    phases["update_gbs"] = round(prof.bytes_update / (upd_ms * 1e-3) / 1e9, 1) if upd_ms else None
-    phases["hbm_peak_gbs"] = hbm
-    phases["kernel_launches_per_step"] = prof.kernel_launches
 
     out = {
         "metric": METRIC, "value": round(ms, 4), "unit": "ms/step", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": cfg["compute"], "data": "synthetic",
-        "config": {"workload": args.workload, "description": cfg["desc"], "matrices": len(specs),
-                   "cuda_graph": bool(args.graph),
-                   "elements": elems, "state_bytes": 12 * elems,
-                   "l2": "inputs larger than L2 (fp32 W, M, G resident in HBM)",
-                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "config": config_for(args, specs),
         "roofline": roof,
         "phases": phases,
+        "normuon_on": normuon_on,
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,
         "device_status": mu.status_str(status),
-        "cuda_graph": bool(args.graph),
         "gemm": "cta_pair" if args.cta_pair else "single_cta",
     }
     return out
@@ -484,8 +618,7 @@ def run_spectrum(args, rank, world, local_rank):
         "metric": METRIC, "value": g["ms"], "unit": "ms/step", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": g["ms"], "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": {"workload": args.workload, "description": cfg["desc"], "step": "one gram_ns_polar call",
-                   "l2": f"bf16 input {2 * n * m / 2**20:.0f} MiB plus working set, larger than L2"},
+        "config": config_for(args),
         "roofline": {"bound": "tensor", "kernel": "gemm_kernel (Gram NS chain)", "achieved": g["tflops_algorithmic"],
                      "peak": peak, "unit": "TFLOP/s", "frac": round(g["tflops_algorithmic"] / peak, 4),
                      "traffic": None, "peak_source": f"{kind} burst bf16 (fp16 has the same dense rate)"},
@@ -501,16 +634,64 @@ def run_spectrum(args, rank, world, local_rank):
 # ---------------------------------------------------------------------------
 
 
-_SAMPLE_INPUTS = {}  # seeded oracle inputs reused by later samples of the same matrix
+class OracleSampler:
+    """Times the fp64 oracle on bounded samples of a layer-set workload.
+
+    Matrices of one shape cost the oracle the same, so the whole step is
+    estimated as each timed shape's mean time times that shape's count. The
+    seeded inputs of every sampled matrix are kept, so later samples of the
+    same matrix do not pay for drawing them again."""
+
+    def __init__(self, workload: str):
+        self.workload = workload
+        self.cfg = WORKLOADS[workload]
+        self.specs = specs_for(workload)
+        self.count = {}
+        self.first = {}
+        for s in self.specs:
+            key = (s.rows, s.cols)
+            self.count[key] = self.count.get(key, 0) + 1
+            self.first.setdefault(key, s)
+        self.shapes = list(self.first)
+        self.times = {}
+        self.inputs = {}
+        self.names = []
+
+    def time_spec(self, s) -> float:
+        import oracle
+        cfg = self.cfg
+        state = self.inputs.get(s.name)
+        if state is None:
+            state = self.inputs[s.name] = host_state(s, self.workload)
+        W, M, G = state
+        v = np.zeros(s.rows, np.float32)
+        p = oracle.StepParams(mu=0.95, lr=0.02, coeffs=(COEFFS,) * 5, gram=cfg["gram"], normuon=cfg["normuon"])
+        if cfg["dion3"] is not None:
+            p = oracle.StepParams(**{**p.__dict__, "k": oracle.rows_for_fraction(s.rows, *cfg["dion3"])})
+        t = time.perf_counter()
+        oracle.muon_step(W, M, G, v, p)
+        dt = time.perf_counter() - t
+        self.times.setdefault((s.rows, s.cols), []).append(dt)
+        self.names.append(s.name)
+        return dt
+
+    def time_shape(self, i: int) -> float:
+        return self.time_spec(self.first[self.shapes[i % len(self.shapes)]])
+
+    def estimate_ms(self) -> float:
+        return 1e3 * sum(float(np.mean(self.times[k])) * self.count[k] for k in self.shapes)
+
+    def describe(self, what: str) -> str:
+        per = ", ".join(f"{r}x{c}: {len(self.times.get((r, c), []))} timed, x{self.count[(r, c)]}"
+                        for (r, c) in self.shapes)
+        return (f"oracle muon_step, {what}; the step is each shape's mean time times its count ({per}); "
+                f"{len(self.specs)} matrices in the step")
 
 
-def oracle_sample(workload: str, budget_s: float):
-    """Time the oracle on a bounded sample of the workload; returns
-    (ms per full step, description of the sample, threads used)."""
+def spectrum_sample(workload: str):
+    """Oracle Gram NS on a scaled-down matrix of the same kind, scaled to the
+    full matrix by the Gram FLOP formula; returns (ms, description)."""
     import oracle
-
-    cfg = WORKLOADS[workload]
-    specs = specs_for(workload)
     if workload == "moe_alpha8_2048x16384":
         X = inputs.gaussian((512, 4096), 1.0, 6000, 0).astype(np.float64)
         t = time.perf_counter()
@@ -518,56 +699,36 @@ def oracle_sample(workload: str, budget_s: float):
         dt = time.perf_counter() - t
         scale = ns_flops(2048, 16384, 5, True) / ns_flops(512, 4096, 5, True)
         return 1e3 * dt * scale, (f"oracle gram_newton_schulz on a 512x4096 Gaussian matrix (aspect 8), "
-                                  f"{dt:.2f} s, scaled x{scale:.0f} by the Gram FLOP formula"), threads_used()
-    if workload == "spectrum4096x16384":
-        t = time.perf_counter()
-        X, _ = inputs.spectrum_matrix(1024, 4096, -4.0, seed=3000)
-        t_gen = time.perf_counter() - t
-        t = time.perf_counter()
-        oracle.gram_newton_schulz(X, (COEFFS,) * 5, 1e-7, 3)
-        dt = time.perf_counter() - t
-        scale = ns_flops(4096, 16384, 5, True) / ns_flops(1024, 4096, 5, True)
-        return 1e3 * dt * scale, (f"oracle gram_newton_schulz on a 1024x4096 matrix of the same spectrum, "
-                                  f"{dt:.1f} s, scaled x{scale:.0f} by the Gram FLOP formula"), threads_used()
-    sp = oracle.StepParams(mu=0.95, lr=0.02, coeffs=(COEFFS,) * 5, gram=cfg["gram"], normuon=cfg["normuon"])
-    # Matrices of one shape cost the oracle the same, so the whole step is
-    # the mean time of each timed shape times that shape's count. One matrix
-    # of every distinct shape is timed first, then more until the budget is
-    # used.
-    count = {}
-    for s in specs:
-        count[(s.rows, s.cols)] = count.get((s.rows, s.cols), 0) + 1
-    seen, first, rest = set(), [], []
-    for i, s in enumerate(specs):
-        (rest if (s.rows, s.cols) in seen else first).append(i)
-        seen.add((s.rows, s.cols))
-    times, names, t_sum = {}, [], 0.0
-    for j, i in enumerate(first + rest):
-        s = specs[i]
-        key = (workload, s.name)
-        state = _SAMPLE_INPUTS.get(key)
-        if state is None:
-            state = host_state(s, workload)
-            if s.rows * s.cols <= (1 << 24):  # keep only moderate matrices across steps
-                _SAMPLE_INPUTS[key] = state
-        W, M, G = state
-        v = np.zeros(s.rows, np.float32)
-        p = sp
-        if cfg["dion3"] is not None:
-            p = oracle.StepParams(**{**sp.__dict__, "k": oracle.rows_for_fraction(s.rows, *cfg["dion3"])})
-        t = time.perf_counter()
-        oracle.muon_step(W, M, G, v, p)
-        dt = time.perf_counter() - t
-        t_sum += dt
-        times.setdefault((s.rows, s.cols), []).append(dt)
-        names.append(s.name)
-        if j + 1 >= len(first) and t_sum > budget_s:
+                                  f"{dt:.2f} s, scaled x{scale:.0f} by the Gram FLOP formula")
+    X, _ = inputs.spectrum_matrix(1024, 4096, -4.0, seed=3000)
+    t = time.perf_counter()
+    oracle.gram_newton_schulz(X, (COEFFS,) * 5, 1e-7, 3)
+    dt = time.perf_counter() - t
+    scale = ns_flops(4096, 16384, 5, True) / ns_flops(1024, 4096, 5, True)
+    return 1e3 * dt * scale, (f"oracle gram_newton_schulz on a 1024x4096 matrix of the same spectrum, "
+                              f"{dt:.1f} s, scaled x{scale:.0f} by the Gram FLOP formula")
+
+
+SPECTRUM = ("spectrum4096x16384", "moe_alpha8_2048x16384")
+
+
+def oracle_baseline(workload: str, budget_s: float):
+    """cpu_baseline of our arm: one matrix of every distinct shape, then more
+    matrices until about budget_s of oracle time. Returns (ms, desc, cores)."""
+    if workload in SPECTRUM:
+        ms, desc = spectrum_sample(workload)
+        return ms, desc, threads_used()
+    smp = OracleSampler(workload)
+    t_sum = 0.0
+    for i in range(len(smp.shapes)):
+        t_sum += smp.time_shape(i)
+    for s in smp.specs:
+        if t_sum > budget_s:
             break
-    est = sum(float(np.mean(ts)) * count[shape] for shape, ts in times.items())
-    desc = (f"oracle muon_step on {len(names)} of {len(specs)} matrices ({', '.join(names[:6])}"
-            f"{', ...' if len(names) > 6 else ''}), {t_sum:.1f} s; the step is each shape's mean time times "
-            f"its count ({len(count)} shapes)")
-    return 1e3 * est, desc, threads_used()
+        if s.name in smp.inputs:
+            continue
+        t_sum += smp.time_spec(s)
+    return smp.estimate_ms(), smp.describe(f"{len(smp.names)} matrices timed in {t_sum:.1f} s"), threads_used()
 
 
 def threads_used():
@@ -578,22 +739,36 @@ def threads_used():
 
 
 def run_reference(args):
-    cfg = WORKLOADS[args.workload]
-    # each step a bounded sample: the whole run stays near 150 s of oracle
-    # time (one matrix of every shape is the least a step times)
-    per_step_budget = max(0.5, 150.0 / max(1, args.steps + args.warmup))
-    for _ in range(args.warmup):
-        oracle_sample(args.workload, per_step_budget)
+    """The reference arm: the fp64 CPU oracle as it stands. Each step (warm-up
+    or timed) times one matrix, the distinct shapes taken in turn, and reports
+    the whole-step estimate from every shape's mean time so far; the warm-up
+    steps (at least one per shape) give every shape a time before the first
+    timed step."""
     vals = []
-    desc = ""
-    for _ in range(args.steps):
-        v, desc, cores = oracle_sample(args.workload, per_step_budget)
-        vals.append(v)
-    ms = float(np.mean(vals))
+    if args.workload in SPECTRUM:
+        for _ in range(args.warmup):
+            spectrum_sample(args.workload)
+        for _ in range(args.steps):
+            ms, desc = spectrum_sample(args.workload)
+            vals.append(ms)
+    else:
+        smp = OracleSampler(args.workload)
+        k = 0
+        for _ in range(max(args.warmup, len(smp.shapes))):
+            smp.time_shape(k)
+            k += 1
+        for _ in range(args.steps):
+            smp.time_shape(k)
+            k += 1
+            vals.append(smp.estimate_ms())
+        desc = smp.describe(f"one matrix per step, shapes in turn, {len(smp.names)} samples")
+    ms = float(np.mean(vals)) if vals else 0.0
+    cfg = WORKLOADS[args.workload]
     return {"impl": "reference", "metric": METRIC, "value": round(ms, 2), "unit": "ms/step", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "description": cfg["desc"]},
+            "config": config_for(args),
+            "reference_precision": f"fp64 oracle of the {cfg['compute']} path",
             "cpu_baseline": {"value": round(ms, 2), "unit": "ms/step", "cores": threads_used(), "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": round(ms, 2), "unit": "ms/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -605,14 +780,17 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt124m")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama7b")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end arm")
-    ap.add_argument("--graph", type=int, default=1, help="1: replay the step as one captured CUDA graph")
+    ap.add_argument("--no-normuon", action="store_true", help="skip the NorMuon-on timing of the Llama-7B set")
+    ap.add_argument("--graph", type=int, default=-1,
+                    help="1: replay the step as one captured CUDA graph, 0: eager with per-step phase events, "
+                         "-1 (default): graph for the small layer sets, eager for the large ones")
     ap.add_argument("--cta-pair", type=int, default=1, help="1: CTA-pair tensor-core GEMM, 0: single-CTA")
     ap.add_argument("--wait-timeout-ms", type=float, default=0.0, help="bound of device-side waits (0: default)")
     args = ap.parse_args()
@@ -638,12 +816,12 @@ def main():
     mu.set_gemm_cta_pair(bool(args.cta_pair))
     if args.wait_timeout_ms > 0:
         mu.set_wait_timeout_ns(int(args.wait_timeout_ms * 1e6))
-    if args.workload in ("spectrum4096x16384", "moe_alpha8_2048x16384"):
+    if args.workload in SPECTRUM:
         out = run_spectrum(args, rank, world, local_rank)
     else:
         out = run_ours(args, rank, world, local_rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        ms, desc, cores = oracle_sample(args.workload, args.cpu_budget)
+        ms, desc, cores = oracle_baseline(args.workload, args.cpu_budget)
         out["cpu_baseline"] = {"value": round(ms, 1), "unit": "ms/step", "cores": cores, "kind": "oracle",
                                "sample": desc}
     if world > 1:

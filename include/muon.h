@@ -268,6 +268,17 @@ typedef struct {
 muon_status muon_step_profiled(const muon_matrix* mats, int32_t count, const muon_params* p,
                                void* ws, size_t ws_bytes, void* stream, muon_step_profile* prof);
 
+/* muon_step that also records five caller-owned CUDA events (cudaEvent_t
+ * handles, created by the caller with timing enabled) on `stream` at the phase
+ * boundaries: events[0] before the first kernel, events[1] before the
+ * Newton-Schulz chain, events[2] after it, events[3] after the NorMuon row
+ * scales, events[4] after the weight update. Same arguments and effects as
+ * muon_step otherwise; it does not synchronise, so a timed loop can measure
+ * each phase of the very steps it times (cudaEventElapsedTime after the
+ * loop). events must be non-NULL and hold five valid events. */
+muon_status muon_step_events(const muon_matrix* mats, int32_t count, const muon_params* p,
+                             void* ws, size_t ws_bytes, void* stream, void* const* events);
+
 /* Number of kernels this library has queued from the calling thread since it
  * was loaded (monotonic; for counting launches inside a timed region). */
 int64_t muon_kernel_launch_count(void);

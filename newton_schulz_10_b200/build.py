@@ -1,7 +1,8 @@
 """Build libmuon.so (all CUDA sources under csrc/) for sm_100a, in-tree.
 
-Usage: python -m newton_schulz_10_b200.build   (or call build()).
-Objects go to newton_schulz_10_b200/_build/, the library next to this file.
+Usage: python -m newton_schulz_10_b200.build [--debug]   (or call build()).
+Objects go to newton_schulz_10_b200/_build/ (_build_check/ for the
+bounds-checked debug build), the library next to this file.
 """
 
 from __future__ import annotations
@@ -15,9 +16,14 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
-BUILD = os.path.join(HERE, "_build")
-LIB = os.path.join(HERE, "libmuon.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
+# normal build, and the bounds-checked debug build (-DMUON_BOUNDS_CHECK):
+# device-side index checks report MUON_ERR_INVALID_ARG through the status word
+VARIANTS = {
+    False: (os.path.join(HERE, "_build"), os.path.join(HERE, "libmuon.so"), []),
+    True: (os.path.join(HERE, "_build_check"), os.path.join(HERE, "libmuon_check.so"), ["-DMUON_BOUNDS_CHECK"]),
+}
+BUILD, LIB, _ = VARIANTS[False]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
@@ -47,10 +53,10 @@ def _stale(obj: str, src: str) -> bool:
     return any(os.path.getmtime(p) > t for p in [src, *_headers()])
 
 
-def _compile(src: str, verbose: bool) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src).replace(".cu", ".o"))
+def _compile(src: str, verbose: bool, build_dir: str, defines) -> str:
+    obj = os.path.join(build_dir, os.path.basename(src).replace(".cu", ".o"))
     if _stale(obj, src):
-        cmd = [nvcc(), *ARCH, *FLAGS, "-c", src, "-o", obj]
+        cmd = [nvcc(), *ARCH, *FLAGS, *defines, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -59,20 +65,24 @@ def _compile(src: str, verbose: bool) -> str:
     return obj
 
 
-def build(verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(verbose: bool = False, debug: bool = False) -> str:
+    """Compile every CUDA source for sm_100a and link the library in-tree.
+    debug=True builds the bounds-checked libmuon_check.so instead (its own
+    object directory; the normal library is untouched)."""
+    build_dir, lib, defines = VARIANTS[bool(debug)]
+    os.makedirs(build_dir, exist_ok=True)
     srcs = _sources()
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
-    if not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", LIB, *objs]
+        objs = list(ex.map(lambda s: _compile(s, verbose, build_dir, defines), srcs))
+    if not os.path.exists(lib) or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
+        cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", lib, *objs]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose="-v" in sys.argv))
+    print(build(verbose="-v" in sys.argv, debug="--debug" in sys.argv))

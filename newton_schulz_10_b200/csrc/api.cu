@@ -282,6 +282,13 @@ StepPlan plan_step(const muon_matrix* mats, int32_t count, const muon_params* p)
   return q;
 }
 
+// True when a (valid) step has no matrix with work: step_impl then queues nothing.
+bool plan_step_empty(const muon_matrix* mats, int32_t count) {
+  for (int i = 0; i < count; ++i)
+    if (mats[i].rows > 0 && mats[i].cols > 0) return false;
+  return true;
+}
+
 muon_status step_impl(const muon_matrix* mats, int32_t count, const muon_params* p, void* ws, size_t ws_bytes,
                       cudaStream_t s, PhaseEvents& E, muon_step_profile* prof) {
   TRY(check_step(mats, count, p));
@@ -632,6 +639,26 @@ muon_status muon_step_profiled(const muon_matrix* mats, int32_t count, const muo
   }
   for (int i = 0; i < 5; ++i) cudaEventDestroy(E.ev[i]);
   return r;
+}
+
+muon_status muon_step_events(const muon_matrix* mats, int32_t count, const muon_params* p, void* ws,
+                             size_t ws_bytes, void* stream, void* const* events) {
+  if (!events) return MUON_ERR_INVALID_ARG;
+  PhaseEvents E;
+  for (int i = 0; i < 5; ++i) {
+    if (!events[i]) return MUON_ERR_INVALID_ARG;
+    E.ev[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  E.on = true;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  muon_status r = step_impl(mats, count, p, ws, ws_bytes, s, E, nullptr);
+  if (r != MUON_OK) return r;
+  // a step with no work still records every event, so the caller's timing
+  // loop never reads an event that was not recorded
+  if (plan_step_empty(mats, count))
+    for (int i = 0; i < 5; ++i)
+      if (cudaEventRecord(E.ev[i], s) != cudaSuccess) return MUON_ERR_CUDA;
+  return MUON_OK;
 }
 
 int64_t muon_kernel_launch_count(void) { return counters().launches; }

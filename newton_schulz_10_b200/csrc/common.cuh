@@ -22,6 +22,21 @@ __device__ __forceinline__ void report(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Debug builds (-DMUON_BOUNDS_CHECK): index checks on the global accesses of
+// the row kernels, the split-K reduction and the GEMM epilogue's C loads. A
+// failed check records MUON_ERR_INVALID_ARG in the status word and the access
+// is skipped; nothing traps. In normal builds every check is `true` and
+// compiles away.
+#ifdef MUON_BOUNDS_CHECK
+__device__ __forceinline__ bool in_bounds(bool ok, int* status) {
+  if (!ok) report(status, MUON_ERR_INVALID_ARG);
+  return ok;
+}
+#define MUON_IN_BOUNDS(cond, status) (::muon::in_bounds((cond), (status)))
+#else
+#define MUON_IN_BOUNDS(cond, status) true
+#endif
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

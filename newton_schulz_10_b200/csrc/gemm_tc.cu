@@ -473,7 +473,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int cr = r0 + 8 * j + (lane >> 2);
-              if (cr < g.M) cv[ch][j] = *reinterpret_cast<const uint4*>(cb + (long long)cr * g.ldc + c0);
+              if (cr < g.M && MUON_IN_BOUNDS(c0 + (lane & 3) * 8 + 8 <= g.ldc, p.status))
+                cv[ch][j] = *reinterpret_cast<const uint4*>(cb + (long long)cr * g.ldc + c0);
             }
           }
         }
@@ -656,6 +657,7 @@ struct SplitGroup {
 struct SplitParams {
   SplitGroup g[kMaxGemmGroups];
   int ngroups;
+  int* status;  // index checks of the bounds-checked build report here
 };
 
 constexpr int RED_THREADS = 256;  // one 32x32 block: 32 rows x 8 groups of 4 columns
@@ -679,7 +681,7 @@ __global__ void __launch_bounds__(RED_THREADS) split_reduce_kernel(const __grid_
   const int rr = threadIdx.x >> 3, cg = (threadIdx.x & 7) * 4;  // this thread: row rr, columns cg..cg+3
   const int r = bi * 32 + rr, c = bj * 32 + cg;
   float v[4] = {0.f, 0.f, 0.f, 0.f};
-  if (r < g.n) {
+  if (r < g.n && MUON_IN_BOUNDS(c + 3 < g.ldp && g.splits <= RED_MAX_PARTS, p.status)) {
     // every part's 4 values in flight at once (the rows' padding keeps the
     // 16-byte loads inside the buffer); then summed in part order
     const float* pp = g.part + ((long long)b * g.n + r) * g.ldp + c;
@@ -1080,6 +1082,7 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
   p.ngroups = ng;
   p.total_tiles = total;
   p.status = status;
+  sp.status = status;
   p.timeout_ns = timeout_ns;
 
   Counters& cn = counters();

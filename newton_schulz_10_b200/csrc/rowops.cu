@@ -92,9 +92,10 @@ __global__ void __launch_bounds__(BLOCK) momentum_rows(const __grid_constant__ R
   __shared__ double scratch[32];
   const int task = blockIdx.x * (BLOCK / WG) + threadIdx.x / WG;
   const int l = threadIdx.x % WG;
-  const bool active = task < L.total_tasks;
+  bool active = task < L.total_tasks;
   const RowMat& m = L.m[find_mat(L, active ? task : L.total_tasks - 1)];
   const int64_t r = active ? task - m.task_begin : 0;
+  if (active) active = MUON_IN_BOUNDS(r >= 0 && r < m.rows && (!CAST || m.ldx >= m.cols), L.status);
   double ss = 0.0, sa = 0.0;
   if (active) {
     float* M = m.M + r * m.cols;
@@ -161,9 +162,10 @@ __global__ void __launch_bounds__(BLOCK) row_stats(const __grid_constant__ RowLa
   __shared__ double scratch[32];
   const int task = blockIdx.x * (BLOCK / WG) + threadIdx.x / WG;
   const int l = threadIdx.x % WG;
-  const bool active = task < L.total_tasks;
+  bool active = task < L.total_tasks;
   const RowMat& m = L.m[find_mat(L, active ? task : L.total_tasks - 1)];
   const int64_t r = active ? task - m.task_begin : 0;
+  if (active) active = MUON_IN_BOUNDS(r >= 0 && r < m.rows, L.status);
   double ss = 0.0, sa = 0.0;
   if (active) {
     const S* x = reinterpret_cast<const S*>(m.src) + r * m.cols;
@@ -211,7 +213,9 @@ __global__ void __launch_bounds__(BLOCK) cast_rows(const __grid_constant__ RowLa
   if (task >= L.total_tasks) return;
   const RowMat& m = L.m[find_mat(L, task)];
   const int64_t i = task - m.task_begin;
+  if (!MUON_IN_BOUNDS(i >= 0 && i < m.ntask && m.ldx >= m.cols, L.status)) return;
   const int64_t j = m.idx ? (int64_t)m.idx[i] : i;
+  if (!MUON_IN_BOUNDS(j >= 0 && j < m.rows, L.status)) return;
   const float mult = (m.mult ? *m.mult : 1.f) * m.kappa;
   const S* x = reinterpret_cast<const S*>(m.src) + j * m.cols;
   T* X = reinterpret_cast<T*>(m.X) + i * m.ldx;
@@ -235,9 +239,10 @@ __global__ void __launch_bounds__(BLOCK) normuon_rows(const __grid_constant__ Ro
   __shared__ double scratch[32];
   const int task = blockIdx.x * (BLOCK / WG) + threadIdx.x / WG;
   const int l = threadIdx.x % WG;
-  const bool active = task < L.total_tasks;
+  bool active = task < L.total_tasks;
   const RowMat& m = L.m[find_mat(L, active ? task : L.total_tasks - 1)];
   const int64_t i = active ? task - m.task_begin : 0;
+  if (active) active = MUON_IN_BOUNDS(i >= 0 && i < m.ntask && m.ldx >= m.cols, L.status);
   float acc = 0.f;
   if (active) {
     const T* o = reinterpret_cast<const T*>(m.X) + i * m.ldx;
@@ -266,7 +271,9 @@ __global__ void __launch_bounds__(BLOCK) update_rows(const __grid_constant__ Row
   if (task >= L.total_tasks) break;
   const RowMat& m = L.m[find_mat(L, task)];
   const int64_t i = task - m.task_begin;
+  if (!MUON_IN_BOUNDS(i >= 0 && i < m.ntask && m.ldx >= m.cols, L.status)) continue;
   const int64_t j = m.idx ? (int64_t)m.idx[i] : i;
+  if (!MUON_IN_BOUNDS(j >= 0 && j < m.rows, L.status)) continue;
   const float step = -L.lr * (m.rscale ? m.rscale[i] : 1.f);
   const T* o = reinterpret_cast<const T*>(m.X) + i * m.ldx;
   float* W = m.W + j * m.cols;
@@ -417,13 +424,14 @@ __global__ void __launch_bounds__(SEL_THREADS) select_topk(const double* key, co
         take = e < need_eq;
         ++e;
       }
-      if (take) idx[pos++] = (int32_t)i;
+      if (take && MUON_IN_BOUNDS(pos >= 0 && pos < k, status)) idx[pos++] = (int32_t)i;
     }
   }
   __syncthreads();
   // Frobenius norm of the selected rows, ascending-index order
   double t = 0.0;
-  for (int64_t i = tid; i < k; i += SEL_THREADS) t += rsum[idx[i]];
+  for (int64_t i = tid; i < k; i += SEL_THREADS)
+    if (MUON_IN_BOUNDS(idx[i] >= 0 && idx[i] < n, status)) t += rsum[idx[i]];
   t = block_sum(t, scratch);
   if (tid == 0) {
     if (!isfinite(t)) report(status, MUON_ERR_NONFINITE);

@@ -13,7 +13,10 @@ import os
 from dataclasses import dataclass, field
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libmuon.so")
+# MUON_BOUNDS_CHECK=1 loads the bounds-checked debug build (built by
+# `python -m newton_schulz_10_b200.build --debug`): the same library with
+# device-side index checks that report MUON_ERR_INVALID_ARG.
+LIB_PATH = os.path.join(HERE, "libmuon_check.so" if os.environ.get("MUON_BOUNDS_CHECK") == "1" else "libmuon.so")
 MAX_T = 16
 
 # muon_status
@@ -27,7 +30,7 @@ NORM_L1, NORM_L2 = 0, 1
 EXPORTS = ("muon_set_wait_timeout_ns", "muon_set_gemm_cta_pair", "muon_status_str", "muon_rows_for_fraction", "muon_ns_params_default",
            "muon_ns_workspace_size", "ns_polar", "gram_ns_polar", "normuon_scale", "muon_select_workspace_size",
            "select_rows", "muon_workspace_size", "muon_step", "muon_step_profiled", "muon_kernel_launch_count",
-           "select_rows_noalloc")
+           "select_rows_noalloc", "muon_step_events")
 
 
 class NsParams(C.Structure):
@@ -105,6 +108,8 @@ def lib() -> C.CDLL:
         L.muon_step_profiled.argtypes = [C.POINTER(Matrix), i32, C.POINTER(Params), vp, sz, vp,
                                          C.POINTER(StepProfile)]
         L.muon_step_profiled.restype = i32
+        L.muon_step_events.argtypes = [C.POINTER(Matrix), i32, C.POINTER(Params), vp, sz, vp, C.POINTER(vp)]
+        L.muon_step_events.restype = i32
         L.muon_kernel_launch_count.argtypes = []
         L.muon_kernel_launch_count.restype = i64
         _lib = L
@@ -307,6 +312,16 @@ class Step:
                                         self.ws.numel(), _stream(stream), C.byref(prof))
         _check(code, "muon_step_profiled")
         return prof
+
+    def timed(self, events, stream=None) -> None:
+        """Run the step, recording the five torch.cuda.Event objects in
+        `events` (enable_timing=True) at its phase boundaries on the stream:
+        start, NS chain start, NS chain end, NorMuon end, update end. Does not
+        synchronise."""
+        handles = (C.c_void_p * 5)(*[e.cuda_event for e in events])
+        code = lib().muon_step_events(self._table, len(self.mats), C.byref(self.params), _ptr(self.ws),
+                                      self.ws.numel(), _stream(stream), handles)
+        _check(code, "muon_step_events")
 
     def device_status(self) -> int:
         """Deferred device status of the last step (synchronises)."""
