@@ -133,6 +133,18 @@ void muon_set_wait_timeout_ns(uint64_t ns);
  * applies to launches queued after the call. */
 void muon_set_gemm_cta_pair(int32_t enable);
 
+/* How the Newton-Schulz chain's products are launched: 0 (default) one
+ * persistent launch per product (all shape groups of the call together); 1
+ * the whole chain as one fused persistent launch (or a few, when its
+ * products need more kernel parameters than one launch holds), in which the
+ * tiles of a product wait, matrix by matrix, until the previous product of
+ * the same matrix is in memory (completion counters in the workspace, each
+ * wait bounded like every other device wait), so that products of different
+ * matrices overlap and no launch boundary separates dependent products.
+ * Both give the same results up to fp32 summation order. Process-wide;
+ * applies to calls made after it. */
+void muon_set_gemm_chain(int32_t enable);
+
 /* Human-readable name of a status value (static string, never NULL). */
 const char* muon_status_str(muon_status s);
 
@@ -239,6 +251,48 @@ size_t muon_workspace_size(const muon_matrix* mats, int32_t count, const muon_pa
  * the same shape are batched into shared launches. */
 muon_status muon_step(const muon_matrix* mats, int32_t count, const muon_params* p,
                       void* ws, size_t ws_bytes, void* stream);
+
+/* The step in three parts, for callers that hold each matrix as row shards
+ * on several GPUs and move whole matrices to an owner GPU for the
+ * orthogonalisation ("4. Megabatched Communication": pack the local momentum
+ * shards into one all-to-all, assemble, orthogonalise as a batch, scatter
+ * back). On one GPU, muon_momentum, then muon_orthogonalize, then
+ * muon_apply_update give the same W, M and v as muon_step, bit for bit.
+ *
+ * muon_momentum: the first line of Eq. (1) on every matrix, elementwise:
+ * M <- mu M + G (one rounding, as a fused multiply-add), or M <- M + G when
+ * p->dion3 (Algorithm 4 keeps the decay for the error feedback). Reads M and
+ * G, writes M; W and v are not touched. No workspace. */
+muon_status muon_momentum(const muon_matrix* mats, int32_t count, const muon_params* p, void* stream);
+
+/* muon_orthogonalize: everything between the momentum and the weight update,
+ * on the momentum M as given (muon_momentum already applied): the Frobenius
+ * scale, the Dion3 selection (p->dion3), the Newton-Schulz chain and NorMuon
+ * (p->normuon, Eq. (2); v is updated in place for the orthogonalised rows).
+ * W and G are not read (they may be NULL). Outputs, per matrix i, all
+ * caller-owned device memory:
+ *   O[i]          rows x cols, ld = cols, 16-byte aligned, element type of
+ *                 p->ns.compute (bf16, fp16 or fp32): the orthogonalised row
+ *                 at its stored row position; zero rows where not selected
+ *   row_scale[i]  rows floats: the update's row scale (NorMuon's scale, or 1);
+ *                 0 where not selected
+ *   selected[i]   rows int32 (needed when p->dion3, else may be NULL): 1 for
+ *                 the selected rows, 0 elsewhere
+ * so that the update is W[r,:] -= lr * row_scale[i][r] * O[i][r,:].
+ * ws / ws_bytes: as for muon_step (muon_workspace_size). */
+muon_status muon_orthogonalize(const muon_matrix* mats, int32_t count, const muon_params* p,
+                               void* const* O, float* const* row_scale, int32_t* const* selected,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/* muon_apply_update: the weight update of Eq. (1) from muon_orthogonalize's
+ * outputs (or row shards of them: mats[i] may be a row range of a matrix
+ * whose O, row_scale and selected rows are passed for the same range):
+ * W[r,:] <- W[r,:] - lr * row_scale[i][r] * O[i][r,:] (one rounding), and,
+ * when p->dion3, M[r,:] <- mu M[r,:] for the selected rows, whose W alone
+ * changes. Reads O, row_scale, selected; G and v are not touched. */
+muon_status muon_apply_update(const muon_matrix* mats, int32_t count, const muon_params* p,
+                              const void* const* O, const float* const* row_scale,
+                              const int32_t* const* selected, void* stream);
 
 /* Per-phase timing and work accounting of one step (muon_step_profiled).
  * Times are CUDA-event milliseconds on the call's stream. FLOPs count the

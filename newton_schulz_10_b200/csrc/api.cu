@@ -120,7 +120,7 @@ muon_status row_batches(const std::vector<RowMat>& mats, const RowLaunch& proto,
 // ---------------------------------------------------------------------------
 
 struct PolarPlan {
-  size_t s, xscale, rsum;
+  size_t s, xscale, rsum, ctr;
   GroupBufs g;
   size_t total;
 };
@@ -131,6 +131,7 @@ PolarPlan plan_polar(int64_t rows, int64_t cols, Op t, const muon_ns_params* p) 
   q.s = off; off += kAlign;
   q.xscale = off; off += kAlign;
   q.rsum = off; off += up((size_t)rows * sizeof(double));
+  q.ctr = off; off += up(ns_counter_words(p, 1) * sizeof(unsigned));
   q.total = layout_group(rows, cols, 1, t, p, off, &q.g);
   return q;
 }
@@ -189,7 +190,7 @@ muon_status polar_impl(const void* X, muon_dtype x_dtype, void* O, muon_dtype o_
   g.rho = rho_for(t, n);
   g.part = q.g.part_bytes ? at<float>(ws, q.g.part) : nullptr;
   g.part_bytes = q.g.part_bytes;
-  TRY(ns_run(t, &g, 1, &pp, status, timeout_ns(), s));
+  TRY(ns_run(t, &g, 1, &pp, status, timeout_ns(), s, at<unsigned>(ws, q.ctr)));
   return launch_copy_out(g.X[g.cur], t, pad_ld(cols), O, o_dtype == MUON_F32 ? Op::F32 : Op::BF16, rows, cols,
                          status, s);
 }
@@ -213,10 +214,13 @@ struct StepPlan {
   };
   std::vector<Mat> mats;
   std::vector<Grp> groups;
-  size_t s, xscale, rsum, rkey, rscale, idx, total;
+  size_t s, xscale, rsum, rkey, rscale, idx, ctr, total;
 };
 
-muon_status check_step(const muon_matrix* mats, int32_t count, const muon_params* p) {
+// Which fields of each muon_matrix an entry point reads.
+enum : int { NEED_W = 1, NEED_M = 2, NEED_G = 4, NEED_ALL = 7 };
+
+muon_status check_step(const muon_matrix* mats, int32_t count, const muon_params* p, int need = NEED_ALL) {
   if (!p || count < 0 || (count > 0 && !mats)) return MUON_ERR_INVALID_ARG;
   TRY(check_ns(&p->ns));
   if (!std::isfinite(p->mu) || !std::isfinite(p->lr)) return MUON_ERR_INVALID_ARG;
@@ -231,8 +235,11 @@ muon_status check_step(const muon_matrix* mats, int32_t count, const muon_params
     const muon_matrix& m = mats[i];
     if (m.rows < 0 || m.cols < 0 || m.rows > INT32_MAX || m.cols > INT32_MAX) return MUON_ERR_SHAPE;
     if (m.rows == 0 || m.cols == 0) continue;
-    if (!m.W || !m.M || !m.G || (p->normuon && !m.v)) return MUON_ERR_INVALID_ARG;
-    if (!aligned16(m.W) || !aligned16(m.M) || !aligned16(m.G) || (m.v && (reinterpret_cast<uintptr_t>(m.v) & 3u)))
+    if (((need & NEED_W) && !m.W) || ((need & NEED_M) && !m.M) || ((need & NEED_G) && !m.G) ||
+        (p->normuon && !m.v))
+      return MUON_ERR_INVALID_ARG;
+    if (((need & NEED_W) && !aligned16(m.W)) || ((need & NEED_M) && !aligned16(m.M)) ||
+        ((need & NEED_G) && !aligned16(m.G)) || (m.v && (reinterpret_cast<uintptr_t>(m.v) & 3u)))
       return MUON_ERR_ALIGN;
   }
   return MUON_OK;
@@ -277,6 +284,15 @@ StepPlan plan_step(const muon_matrix* mats, int32_t count, const muon_params* p)
   q.rkey = off; off += up(rows_total * sizeof(double) + 8);
   q.rscale = off; off += up(tasks_total * sizeof(float) + 4);
   q.idx = off; off += up(tasks_total * sizeof(int32_t) + 4);
+  // fused-chain completion counters: each batch of up to kMaxGemmGroups
+  // shape groups runs its own chain, so the largest batch's matrices bound it
+  int64_t chain_mats = 0;
+  for (size_t g0 = 0; g0 < q.groups.size(); g0 += kMaxGemmGroups) {
+    int64_t m = 0;
+    for (size_t gi = g0; gi < q.groups.size() && gi < g0 + kMaxGemmGroups; ++gi) m += q.groups[gi].count;
+    chain_mats = m > chain_mats ? m : chain_mats;
+  }
+  q.ctr = off; off += up(ns_counter_words(&p->ns, chain_mats) * sizeof(unsigned) + 4);
   for (auto& g : q.groups) off = layout_group(g.rows, g.cols, g.count, t, &p->ns, off, &g.b);
   q.total = off;
   return q;
@@ -421,7 +437,7 @@ muon_status step_impl(const muon_matrix* mats, int32_t count, const muon_params*
   E.mark(1, s);
   for (size_t g0 = 0; g0 < ns.size(); g0 += kMaxGemmGroups) {
     const int ng = (int)(ns.size() - g0 < (size_t)kMaxGemmGroups ? ns.size() - g0 : kMaxGemmGroups);
-    TRY(ns_run(t, ns.data() + g0, ng, &p->ns, status, timeout_ns(), s));
+    TRY(ns_run(t, ns.data() + g0, ng, &p->ns, status, timeout_ns(), s, at<unsigned>(ws, q.ctr)));
   }
   E.mark(2, s);
 
@@ -468,6 +484,174 @@ muon_status step_impl(const muon_matrix* mats, int32_t count, const muon_params*
   return MUON_OK;
 }
 
+// The middle of a step, on momentum already updated (muon_orthogonalize):
+// norms / selection, the operand cast, the Newton-Schulz chain and NorMuon,
+// exactly as step_impl computes them, with the orthogonalised rows, their
+// update scales and the selection written to caller buffers.
+muon_status ortho_impl(const muon_matrix* mats, int32_t count, const muon_params* p, void* const* O,
+                       float* const* row_scale, int32_t* const* selected, void* ws, size_t ws_bytes, cudaStream_t s) {
+  TRY(check_step(mats, count, p, NEED_M));
+  if (count > 0 && (!O || !row_scale || (p->dion3 && !selected))) return MUON_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    if (mats[i].rows == 0 || mats[i].cols == 0) continue;
+    if (!O[i] || !row_scale[i] || (p->dion3 && !selected[i])) return MUON_ERR_INVALID_ARG;
+    if (!aligned16(O[i]) || (reinterpret_cast<uintptr_t>(row_scale[i]) & 3u) ||
+        (p->dion3 && (reinterpret_cast<uintptr_t>(selected[i]) & 3u)))
+      return MUON_ERR_ALIGN;
+  }
+  const StepPlan q = plan_step(mats, count, p);
+  if (q.groups.empty()) return MUON_OK;
+  if (!ws) return MUON_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MUON_ERR_ALIGN;
+  if (ws_bytes < q.total) return MUON_ERR_WORKSPACE;
+  Op t;
+  op_of(p->ns.compute, &t);
+  const size_t es = op_size(t);
+  int* status = p->dev_status ? p->dev_status : at<int>(ws, 0);
+  if (!p->dev_status && cudaMemsetAsync(status, 0, sizeof(int), s) != cudaSuccess) return MUON_ERR_CUDA;
+  auto xslot = [&](int i) -> void* {
+    const StepPlan::Mat& e = q.mats[i];
+    const StepPlan::Grp& g = q.groups[e.group];
+    return at<char>(ws, g.b.X[0]) + (size_t)e.gidx * g.rows * pad_ld(g.cols) * es;
+  };
+  // muon_step casts plain-Muon bf16 operands unscaled (the Frobenius scale
+  // enters the first GEMM epilogues); the same here, so the operands agree
+  const bool unscaled = !p->dion3 && t == Op::BF16;
+  RowLaunch proto{};
+  proto.mu = p->mu;
+  proto.lr = p->lr;
+  proto.key_l2 = p->select_norm == MUON_NORM_L2;
+  proto.status = status;
+
+  // 1. row sums of squares and selection keys of the momentum
+  std::vector<RowMat> rm;
+  for (int i = 0; i < count; ++i) {
+    const StepPlan::Mat& e = q.mats[i];
+    if (e.group < 0) continue;
+    RowMat r{};
+    r.src = mats[i].M;
+    r.rows = mats[i].rows;
+    r.cols = mats[i].cols;
+    r.rsum = at<double>(ws, q.rsum) + e.row_base;
+    r.rkey = p->dion3 ? at<double>(ws, q.rkey) + e.row_base : nullptr;
+    r.ntask = (int32_t)mats[i].rows;
+    rm.push_back(r);
+  }
+  TRY(row_batches(rm, proto, [&](RowLaunch& L) { return launch_row_stats(L, Op::F32, s); }));
+
+  // 2. Frobenius scale (+ selection), then the operand cast
+  float* sc = at<float>(ws, q.s);
+  float* xs = at<float>(ws, q.xscale);
+  int32_t* idx = at<int32_t>(ws, q.idx);
+  if (!p->dion3) {
+    std::vector<NormOut> no;
+    for (int i = 0; i < count; ++i) {
+      const StepPlan::Mat& e = q.mats[i];
+      if (e.group < 0) continue;
+      const int64_t n = mats[i].rows < mats[i].cols ? mats[i].rows : mats[i].cols;
+      const int sl = q.groups[e.group].slot0 + e.gidx;
+      no.push_back(NormOut{at<double>(ws, q.rsum) + e.row_base, mats[i].rows, sc + sl, xs + sl,
+                           unscaled ? -1.f : 1.f / kappa_for(t, n)});
+    }
+    TRY(launch_norm_finalize(no.data(), (int)no.size(), p->ns.norm_eps, status, s));
+  } else {
+    for (int i = 0; i < count; ++i) {
+      const StepPlan::Mat& e = q.mats[i];
+      if (e.group < 0) continue;
+      const int64_t n = e.rows_eff < mats[i].cols ? e.rows_eff : mats[i].cols;
+      const int sl = q.groups[e.group].slot0 + e.gidx;
+      TRY(launch_select(at<double>(ws, q.rkey) + e.row_base, at<double>(ws, q.rsum) + e.row_base, mats[i].rows,
+                        e.rows_eff, idx + e.task_base, sc + sl, xs + sl, p->ns.norm_eps, 1.f / kappa_for(t, n),
+                        status, s));
+    }
+  }
+  std::vector<RowMat> cm;
+  for (int i = 0; i < count; ++i) {
+    const StepPlan::Mat& e = q.mats[i];
+    if (e.group < 0) continue;
+    const int64_t n = e.rows_eff < mats[i].cols ? e.rows_eff : mats[i].cols;
+    RowMat r{};
+    r.src = mats[i].M;
+    r.X = xslot(i);
+    r.idx = p->dion3 ? idx + e.task_base : nullptr;
+    r.mult = unscaled ? nullptr : sc + q.groups[e.group].slot0 + e.gidx;
+    r.kappa = unscaled ? 1.f : kappa_for(t, n);
+    r.rows = mats[i].rows;
+    r.cols = mats[i].cols;
+    r.ldx = pad_ld(mats[i].cols);
+    r.ntask = (int32_t)e.rows_eff;
+    cm.push_back(r);
+  }
+  TRY(row_batches(cm, proto, [&](RowLaunch& L) { return launch_cast_rows(L, Op::F32, t, s); }));
+
+  // 3. Newton-Schulz
+  std::vector<NsGroup> ns(q.groups.size());
+  for (size_t gi = 0; gi < q.groups.size(); ++gi) {
+    const StepPlan::Grp& g = q.groups[gi];
+    NsGroup& n = ns[gi];
+    n.rows = g.rows;
+    n.cols = g.cols;
+    n.count = g.count;
+    n.X[0] = at<void>(ws, g.b.X[0]);
+    n.X[1] = at<void>(ws, g.b.X[1]);
+    n.cur = 0;
+    for (int k = 0; k < ns_work_buffers(&p->ns); ++k) n.nb[k] = at<void>(ws, g.b.nb[k]);
+    n.rho = rho_for(t, g.rows < g.cols ? g.rows : g.cols);
+    n.part = g.b.part_bytes ? at<float>(ws, g.b.part) : nullptr;
+    n.part_bytes = g.b.part_bytes;
+    n.xscale = xs + g.slot0;
+  }
+  for (size_t g0 = 0; g0 < ns.size(); g0 += kMaxGemmGroups) {
+    const int ng = (int)(ns.size() - g0 < (size_t)kMaxGemmGroups ? ns.size() - g0 : kMaxGemmGroups);
+    TRY(ns_run(t, ns.data() + g0, ng, &p->ns, status, timeout_ns(), s, at<unsigned>(ws, q.ctr)));
+  }
+
+  // 4. NorMuon row scales, 5. the rows, scales and selection to the caller
+  float* rscale = at<float>(ws, q.rscale);
+  std::vector<RowMat> um;
+  for (int i = 0; i < count; ++i) {
+    const StepPlan::Mat& e = q.mats[i];
+    if (e.group < 0) continue;
+    const StepPlan::Grp& g = q.groups[e.group];
+    RowMat r{};
+    r.v = mats[i].v;
+    r.X = static_cast<char*>(ns[e.group].X[ns[e.group].cur]) + (size_t)e.gidx * g.rows * pad_ld(g.cols) * es;
+    r.ldx = pad_ld(mats[i].cols);
+    r.idx = p->dion3 ? idx + e.task_base : nullptr;
+    r.rscale = p->normuon ? rscale + e.task_base : nullptr;
+    r.out = O[i];
+    r.out_scale = row_scale[i];
+    r.out_flag = p->dion3 ? selected[i] : nullptr;
+    r.rows = mats[i].rows;
+    r.cols = mats[i].cols;
+    r.ntask = (int32_t)e.rows_eff;
+    um.push_back(r);
+  }
+  if (p->normuon) {
+    TRY(row_batches(um, proto, [&](RowLaunch& L) { return launch_normuon_rows(L, t, s); }));
+    std::vector<NormuonMat> nm;
+    for (int i = 0; i < count; ++i) {
+      const StepPlan::Mat& e = q.mats[i];
+      if (e.group < 0) continue;
+      nm.push_back(NormuonMat{rscale + e.task_base, e.rows_eff, mats[i].cols, mats[i].v,
+                              p->dion3 ? idx + e.task_base : nullptr});
+    }
+    TRY(launch_normuon_finalize_batched(nm.data(), (int)nm.size(), p->beta2, p->normuon_eps, status, s));
+  }
+  if (p->dion3) {
+    // rows that are not selected: zero update, scale 0, flag 0
+    for (int i = 0; i < count; ++i) {
+      if (q.mats[i].group < 0) continue;
+      const size_t rows = (size_t)mats[i].rows;
+      if (cudaMemsetAsync(O[i], 0, rows * mats[i].cols * es, s) != cudaSuccess ||
+          cudaMemsetAsync(row_scale[i], 0, rows * sizeof(float), s) != cudaSuccess ||
+          cudaMemsetAsync(selected[i], 0, rows * sizeof(int32_t), s) != cudaSuccess)
+        return MUON_ERR_CUDA;
+    }
+  }
+  return row_batches(um, proto, [&](RowLaunch& L) { return launch_scatter_rows(L, t, s); });
+}
+
 }  // namespace
 }  // namespace muon
 
@@ -478,6 +662,8 @@ extern "C" {
 void muon_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns ? ns : kDefaultTimeoutNs); }
 
 void muon_set_gemm_cta_pair(int32_t enable) { set_gemm_pair_mode(enable ? 2 : 1); }
+
+void muon_set_gemm_chain(int32_t enable) { set_gemm_chain(enable); }
 
 const char* muon_status_str(muon_status s) {
   switch (s) {
@@ -659,6 +845,69 @@ muon_status muon_step_events(const muon_matrix* mats, int32_t count, const muon_
     for (int i = 0; i < 5; ++i)
       if (cudaEventRecord(E.ev[i], s) != cudaSuccess) return MUON_ERR_CUDA;
   return MUON_OK;
+}
+
+muon_status muon_momentum(const muon_matrix* mats, int32_t count, const muon_params* p, void* stream) {
+  TRY(check_step(mats, count, p, NEED_M | NEED_G));
+  std::vector<RowMat> rm;
+  for (int i = 0; i < count; ++i) {
+    if (mats[i].rows == 0 || mats[i].cols == 0) continue;
+    RowMat r{};
+    r.M = mats[i].M;
+    r.G = mats[i].G;
+    r.rows = mats[i].rows;
+    r.cols = mats[i].cols;
+    r.ntask = (int32_t)mats[i].rows;
+    rm.push_back(r);
+  }
+  RowLaunch proto{};
+  proto.mu = p->mu;
+  proto.mode = p->dion3 ? MOM_DION3 : MOM_MUON;
+  proto.status = p->dev_status;
+  Op t;
+  op_of(p->ns.compute, &t);
+  return row_batches(rm, proto, [&](RowLaunch& L) {
+    return launch_momentum_rows(L, t, static_cast<cudaStream_t>(stream));
+  });
+}
+
+muon_status muon_orthogonalize(const muon_matrix* mats, int32_t count, const muon_params* p, void* const* O,
+                               float* const* row_scale, int32_t* const* selected, void* ws, size_t ws_bytes,
+                               void* stream) {
+  return ortho_impl(mats, count, p, O, row_scale, selected, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+muon_status muon_apply_update(const muon_matrix* mats, int32_t count, const muon_params* p, const void* const* O,
+                              const float* const* row_scale, const int32_t* const* selected, void* stream) {
+  TRY(check_step(mats, count, p, NEED_W | (p && p->dion3 ? NEED_M : 0)));
+  if (count > 0 && (!O || !row_scale || (p->dion3 && !selected))) return MUON_ERR_INVALID_ARG;
+  Op t;
+  op_of(p->ns.compute, &t);
+  std::vector<RowMat> um;
+  for (int i = 0; i < count; ++i) {
+    if (mats[i].rows == 0 || mats[i].cols == 0) continue;
+    if (!O[i] || !row_scale[i] || (p->dion3 && !selected[i])) return MUON_ERR_INVALID_ARG;
+    if (!aligned16(O[i])) return MUON_ERR_ALIGN;
+    RowMat r{};
+    r.W = mats[i].W;
+    r.M = mats[i].M;
+    r.X = const_cast<void*>(O[i]);
+    r.ldx = mats[i].cols;
+    r.rscale = const_cast<float*>(row_scale[i]);
+    r.flag = p->dion3 ? selected[i] : nullptr;
+    r.rows = mats[i].rows;
+    r.cols = mats[i].cols;
+    r.ntask = (int32_t)mats[i].rows;
+    um.push_back(r);
+  }
+  RowLaunch proto{};
+  proto.mu = p->mu;
+  proto.lr = p->lr;
+  proto.mode = p->dion3 ? 1 : 0;
+  proto.status = p->dev_status;
+  return row_batches(um, proto, [&](RowLaunch& L) {
+    return launch_update_rows(L, t, static_cast<cudaStream_t>(stream));
+  });
 }
 
 int64_t muon_kernel_launch_count(void) { return counters().launches; }

@@ -46,6 +46,7 @@
 // copies and MMAs are drained with bounded waits (for a pair, by counting
 // what each producer issued: settle_pair_copies) and TMEM is freed before the
 // CTA exits.
+#include <algorithm>
 #include <atomic>
 #include <cstring>
 #include <mutex>
@@ -85,11 +86,14 @@ struct Cfg {
   static_assert(SMEM <= 232448, "exceeds the opt-in shared memory of one sm_100 CTA");
 };
 
-struct Group {
-  CUtensorMap tmA;
-  CUtensorMap tmB;
-  CUtensorMap tmD;  // 32x32 boxes, 64-byte swizzle: epilogue stores
-  CUtensorMap tmP;  // split K: fp32 partials [splits*batch][M][ldp], 32x32 boxes, 128-byte swizzle
+// Distinct tensor maps of one launch, and the jobs of one launch. A job is
+// one product of one shape group (all its matrices); a standalone launch
+// holds up to kMaxGemmGroups jobs, a fused chain launch the products of a
+// whole Newton-Schulz chain, phase after phase.
+constexpr int kMaxMaps = 48;
+constexpr int kMaxJobs = 72;
+
+struct Job {
   void* D;
   const void* C;
   const float* scale;
@@ -100,15 +104,26 @@ struct Group {
   float alpha, beta, gamma;
   int tiles_m, tiles_n, tiles_per_batch, tile_begin;  // tiles_per_batch counts (tile, split) units
   int splits, kbps;                                    // K split in parts of kbps k-blocks (1, all)
+  int mA, mB, mD, mP;  // tensor maps: operands, output (32x32 boxes, 64-byte swizzle), split-K partials
+  // fused chain: counters[done + b] counts the epilogue warps that finished
+  // a tile of matrix b of this job; the job's tiles of matrix b wait until
+  // counters[dep + b] reaches dep_target (the previous product of the same
+  // matrix is complete). -1: no counter / no wait.
+  int done, dep;
+  unsigned dep_target;
 };
 
 struct Params {
-  Group g[kMaxGemmGroups];
-  int ngroups;
+  CUtensorMap maps[kMaxMaps];
+  Job g[kMaxJobs];
+  int ngroups;  // jobs
+  int nmaps;
   int total_tiles;
+  unsigned* counters;  // fused chain only
   int* status;
   unsigned long long timeout_ns;
 };
+static_assert(sizeof(Params) <= 32764, "kernel parameters are limited to 32764 bytes");
 
 struct Tile {
   int g, b, m0, n0;  // m0: first row of the (pair) tile
@@ -124,9 +139,13 @@ __host__ __device__ inline int sym_row_tiles(int i, int tiles_n, int tile_m, int
 
 template <int PAIR, int BN>
 __device__ inline Tile decode(const Params& p, int tile) {
-  int gi = 0;
-  while (gi + 1 < p.ngroups && tile >= p.g[gi + 1].tile_begin) ++gi;
-  const Group& g = p.g[gi];
+  int lo = 0, hi = p.ngroups - 1;  // the last job whose first tile is <= tile
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.g[mid].tile_begin <= tile) lo = mid; else hi = mid - 1;
+  }
+  const int gi = lo;
+  const Job& g = p.g[gi];
   int local = tile - g.tile_begin;
   int b = local / g.tiles_per_batch;
   int t = local - b * g.tiles_per_batch;
@@ -185,6 +204,43 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, int* 
       break;
     }
   }
+}
+
+// Fused chain: completion counters in global memory. A finished tile's
+// stores are complete (bulk_wait0) and fenced for the async proxy before the
+// release increment; a waiter's acquire load is followed by a proxy fence
+// before its tensor copies read the data.
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* a) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(unsigned* a, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// Wait (bounded by budget) until matrix b of the job this one depends on is
+// complete. Returns false when another role raised *abort, or on expiry, in
+// which case it raises *abort and records MUON_ERR_TIMEOUT.
+__device__ __forceinline__ bool wait_dep(const Params& p, const Job& g, int b, volatile int* abort, uint64_t budget) {
+  if (g.dep < 0) return true;
+  const unsigned* c = p.counters + g.dep + b;
+  if (ld_acquire_gpu(c) < g.dep_target) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+      __nanosleep(100);
+      if (ld_acquire_gpu(c) >= g.dep_target) break;
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > budget) {
+        *abort = 1;
+        report(p.status, MUON_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+  fence_proxy_async_global();
+  return true;
 }
 
 // CTA-pair early exit: wait until every operand copy that either CTA issued
@@ -275,12 +331,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     }
   }
   if (warp == 0 && lane == 0) {
-    for (int i = 0; i < p.ngroups; ++i) {
-      prefetch_tmap(&p.g[i].tmA);
-      prefetch_tmap(&p.g[i].tmB);
-      prefetch_tmap(&p.g[i].tmD);
-      if (p.g[i].splits > 1) prefetch_tmap(&p.g[i].tmP);
-    }
+    for (int i = 0; i < p.nmaps; ++i) prefetch_tmap(&p.maps[i]);
   }
   tc_fence_before();
   __syncwarp();
@@ -308,10 +359,16 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     int issued = 0;
     for (int tile = unit; tile < p.total_tiles; tile += units) {
       const Tile t = decode<PAIR, BN>(p, tile);
-      const Group& g = p.g[t.g];
+      const Job& g = p.g[t.g];
+      const CUtensorMap* mapA = &p.maps[g.mA];
+      const CUtensorMap* mapB = &p.maps[g.mB];
       const int am0 = t.m0 + (int)rank * BM;            // this CTA's rows of A
       const int bn0 = t.n0 + (int)rank * (BN / PAIR);   // this CTA's rows of B
       bool ok = true;
+      if (!wait_dep(p, g, t.b, abort_flag, budget)) {
+        raise_peer();
+        break;
+      }
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
         if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, budget, p.status)) {
           raise_peer();
@@ -328,17 +385,17 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         };
         if (issues_a) {
           if (!g.a_mn) {
-            load(a, &g.tmA, k0, am0);
+            load(a, mapA, k0, am0);
           } else {
-            load(a, &g.tmA, am0, k0);
-            load(a + 8192, &g.tmA, am0 + 64, k0);
+            load(a, mapA, am0, k0);
+            load(a + 8192, mapA, am0 + 64, k0);
           }
         } else {
           if (!g.b_mn) {
-            load(b, &g.tmB, k0, bn0);
+            load(b, mapB, k0, bn0);
           } else {
 #pragma unroll
-            for (int j = 0; j < BN / PAIR / 64; ++j) load(b + j * 8192, &g.tmB, bn0 + 64 * j, k0);
+            for (int j = 0; j < BN / PAIR / 64; ++j) load(b + j * 8192, mapB, bn0 + 64 * j, k0);
           }
         }
         ++issued;
@@ -380,7 +437,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     bool ok = true;
     for (int tile = unit; tile < p.total_tiles && ok; tile += units) {
       const Tile t = decode<PAIR, BN>(p, tile);
-      const Group& g = p.g[t.g];
+      const Job& g = p.g[t.g];
       const uint32_t idesc = idesc_f16(fmt, g.a_mn, g.b_mn, BM * PAIR, BN);
       // K-major: 8-row groups 1024 B apart, one K step = 32 B inside the
       // swizzle atom. MN-major: 64-element MN atoms 8 KB apart (LBO), 8-row
@@ -450,7 +507,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     uint32_t acc_phase = 0;
     for (int tile = unit; tile < p.total_tiles; tile += units) {
       const Tile t = decode<PAIR, BN>(p, tile);
-      const Group& g = p.g[t.g];
+      const Job& g = p.g[t.g];
       const float s = g.scale ? g.scale[t.b] : 1.f;
       const float alpha = g.alpha * powi(s, g.alpha_pow);
       const float beta = g.beta * powi(s, g.beta_pow);
@@ -464,6 +521,18 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       uint4 cv[EPI_CHUNKS][4];
       const bool part = g.splits > 1;  // store the raw fp32 partial accumulator
       const bool want_c = g.beta != 0.f && !part;  // warp-uniform
+      if (want_c && g.dep >= 0) {
+        // C was written by an earlier product of the chain: wait for it here
+        // too (these loads are issued before this tile's MMAs complete)
+        bool dok = true;
+        if (lane == 0) dok = wait_dep(p, g, t.b, abort_flag, budget);
+        dok = __shfl_sync(0xffffffffu, dok, 0);
+        __syncwarp();  // the other lanes' loads below are ordered after lane 0's acquire
+        if (!dok) {
+          if (lane == 0) raise_peer();
+          break;
+        }
+      }
       if (want_c) {
         const T* cb = reinterpret_cast<const T*>(g.C) + (long long)t.b * g.sC + (lane & 3) * 8;
 #pragma unroll
@@ -474,7 +543,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
             for (int j = 0; j < 4; ++j) {
               const int cr = r0 + 8 * j + (lane >> 2);
               if (cr < g.M && MUON_IN_BOUNDS(c0 + (lane & 3) * 8 + 8 <= g.ldc, p.status))
-                cv[ch][j] = *reinterpret_cast<const uint4*>(cb + (long long)cr * g.ldc + c0);
+                cv[ch][j] = __ldcg(reinterpret_cast<const uint4*>(cb + (long long)cr * g.ldc + c0));
             }
           }
         }
@@ -508,7 +577,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
           fence_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_3d(&g.tmP, smem_u32(sd), c0, r0, t.split * g.batch + t.b);
+            tma_store_3d(&p.maps[g.mP], smem_u32(sd), c0, r0, t.split * g.batch + t.b);
             bulk_commit();
           }
           continue;
@@ -596,8 +665,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         fence_async_smem();  // generic-proxy writes become visible to the bulk copy
         __syncwarp();
         if (lane == 0) {
-          tma_store_3d(&g.tmD, smem_u32(sd), c0, r0, t.b);
-          if (mirror) tma_store_3d(&g.tmD, smem_u32(sm), r0, c0, t.b);
+          tma_store_3d(&p.maps[g.mD], smem_u32(sd), c0, r0, t.b);
+          if (mirror) tma_store_3d(&p.maps[g.mD], smem_u32(sm), r0, c0, t.b);
           bulk_commit();
         }
       }
@@ -608,6 +677,12 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       if (lane == 0) {
         if (PAIR == 2 && rank != 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[acc]), 0));
         else mbar_arrive(&tempty[acc]);
+        if (g.done >= 0) {
+          // fused chain: this warp's share of the tile is in global memory
+          bulk_wait0();
+          fence_proxy_async_global();
+          red_release_gpu_add(p.counters + g.done + t.b, 1u);
+        }
       }
       if (++acc == 2) {
         acc = 0;
@@ -921,6 +996,12 @@ int num_sms() {
 
 void set_gemm_pair_mode(int pair) { g_pair_mode = pair == 1 ? 1 : 2; }
 
+namespace {
+int g_chain_mode = 0;
+}
+void set_gemm_chain(int on) { g_chain_mode = on ? 1 : 0; }
+int gemm_chain() { return g_chain_mode; }
+
 size_t tc_split_scratch(int64_t n, int64_t K, int count) {
   size_t best = 0;
   const int nkb = (int)((K + tc::BK - 1) / tc::BK);
@@ -950,6 +1031,104 @@ muon_status launch_for(Op t, int pair, const tc::Params& p, int total, int units
   return t == Op::BF16 ? launch<__nv_bfloat16, 1, BN>(p, total, units, s) : launch<__half, 1, BN>(p, total, units, s);
 }
 
+namespace {
+
+// Tensor maps of one launch, each distinct map once (a fused chain reuses
+// the same few buffers in many products).
+struct MapTable {
+  struct Key {
+    const void* base;
+    int64_t inner, outer, batch, ld, bstride;
+    int box_outer, box_inner, swz, dt;
+    bool operator==(const Key& o) const {
+      return base == o.base && inner == o.inner && outer == o.outer && batch == o.batch && ld == o.ld &&
+             bstride == o.bstride && box_outer == o.box_outer && box_inner == o.box_inner && swz == o.swz &&
+             dt == o.dt;
+    }
+  };
+  tc::Params* p;
+  Key keys[tc::kMaxMaps];
+  // Index of the map (made on first use); -1 if it cannot be made or the
+  // table is full.
+  int get(Op t, const void* base, int64_t inner, int64_t outer, int64_t batch, int64_t ld, int64_t bstride,
+          int box_outer, int box_inner = 64, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+    const Key k{base, inner, outer, batch, ld, bstride, box_outer, box_inner, (int)swz, (int)t};
+    for (int i = 0; i < p->nmaps; ++i)
+      if (keys[i] == k) return i;
+    if (p->nmaps >= tc::kMaxMaps) return -1;
+    if (!make_map(&p->maps[p->nmaps], t, base, inner, outer, batch, ld, bstride, box_outer, box_inner, swz)) return -1;
+    keys[p->nmaps] = k;
+    return p->nmaps++;
+  }
+};
+
+// Tensor maps and scalars of one job at tile width bn, K in `parts` parts of
+// `kbps` k-blocks. Returns false if a map cannot be made or the table is full.
+bool fill_job(tc::Job& g, const GemmDesc& d, Op t, int pair, int bn, int parts, int kbps, MapTable& mt) {
+  const int tile_m = tc::BM * pair;
+  // A operand source: K-major [M][K], MN-major [K][M]; 128 rows per CTA.
+  // B operand source: K-major [N][K], MN-major [K][N]; bn / pair rows per CTA.
+  g.mA = d.a_mn ? mt.get(t, d.A, d.M, d.K, d.batch, d.lda, d.strideA, 64)
+                : mt.get(t, d.A, d.K, d.M, d.batch, d.lda, d.strideA, tc::BM);
+  g.mB = d.b_mn ? mt.get(t, d.B, d.N, d.K, d.batch, d.ldb, d.strideB, 64)
+                : mt.get(t, d.B, d.K, d.N, d.batch, d.ldb, d.strideB, bn / pair);
+  g.mD = mt.get(t, d.D, d.N, d.M, d.batch, d.ldd, d.strideD, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  g.mP = -1;
+  if (parts > 1) {
+    const int64_t ldp = pad_ld(d.N);
+    g.mP = mt.get(Op::F32, d.part, d.N, d.M, (int64_t)parts * d.batch, ldp, (int64_t)d.M * ldp, 32, 32);
+    if (g.mP < 0) return false;
+  }
+  if (g.mA < 0 || g.mB < 0 || g.mD < 0) return false;
+  g.D = d.D;
+  g.C = d.C;
+  g.scale = d.scale;
+  g.ldd = d.ldd;
+  g.sD = d.strideD;
+  g.ldc = d.ldc;
+  g.sC = d.strideC;
+  g.M = d.M;
+  g.N = d.N;
+  g.K = d.K;
+  g.batch = d.batch;
+  g.a_mn = d.a_mn;
+  g.b_mn = d.b_mn;
+  g.sym = d.sym;
+  g.alpha_pow = d.alpha_pow;
+  g.beta_pow = d.beta_pow;
+  g.alpha = d.alpha;
+  g.beta = d.beta;
+  g.gamma = d.gamma;
+  g.tiles_m = (d.M + tile_m - 1) / tile_m;
+  g.tiles_n = (d.N + bn - 1) / bn;
+  g.tiles_per_batch = desc_tiles(d, tile_m, bn) * parts;
+  g.splits = parts;
+  g.kbps = kbps;
+  g.done = -1;
+  g.dep = -1;
+  g.dep_target = 0;
+  return true;
+}
+
+muon_status check_desc(const GemmDesc& d) {
+  if (d.ldd % 64 || (d.beta != 0.f && d.ldc % 64)) return MUON_ERR_INVALID_ARG;
+  if (d.sym && d.M != d.N) return MUON_ERR_INVALID_ARG;
+  return MUON_OK;
+}
+
+bool has_work(const GemmDesc& d) { return d.batch > 0 && d.M > 0 && d.N > 0 && d.K > 0; }
+
+// Work accounting of one job (dense, symmetric-once and executed FLOPs).
+void count_job(const tc::Job& g, int tile_m, int bn) {
+  Counters& cn = counters();
+  const double mnk = (double)g.M * g.N * g.K * g.batch;
+  cn.flops_dense += 2.0 * mnk;
+  cn.flops_sym += g.sym ? mnk : 2.0 * mnk;
+  cn.flops_exec += 2.0 * tile_m * bn * (double)g.K * (g.tiles_per_batch / g.splits) * g.batch;
+}
+
+}  // namespace
+
 muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t timeout_ns, cudaStream_t s) {
   if (ngroups < 1 || ngroups > kMaxGemmGroups || (t != Op::BF16 && t != Op::F16)) return MUON_ERR_INVALID_ARG;
   const int pair = g_pair_mode;
@@ -964,9 +1143,9 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
   int ng = 0, total_wide = 0;
   for (int i = 0; i < ngroups; ++i) {
     const GemmDesc& d = gd[i];
-    if (d.batch <= 0 || d.M <= 0 || d.N <= 0 || d.K <= 0) continue;
-    if (d.ldd % 64 || (d.beta != 0.f && d.ldc % 64)) return MUON_ERR_INVALID_ARG;
-    if (d.sym && d.M != d.N) return MUON_ERR_INVALID_ARG;
+    if (!has_work(d)) continue;
+    const muon_status c = check_desc(d);
+    if (c != MUON_OK) return c;
     src[ng++] = &d;
     total_wide += desc_tiles(d, tile_m, tc::BN_WIDE) * d.batch;
   }
@@ -1000,58 +1179,24 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
     }
   }
 
-  tc::Params p;
+  static thread_local tc::Params p;  // ~20 KB: kept off the stack
   memset(&p, 0, sizeof(p));
+  static thread_local MapTable mt;
+  mt.p = &p;
   tc::SplitParams sp;
   memset(&sp, 0, sizeof(sp));
-  int base_tiles[kMaxGemmGroups];
   int red_blocks = 0;
   for (int i = 0; i < ng; ++i) {
     const GemmDesc& d = *src[i];
-    tc::Group& g = p.g[i];
-    // A operand source: K-major [M][K], MN-major [K][M]; 128 rows per CTA.
-    // B operand source: K-major [N][K], MN-major [K][N]; bn / pair rows per CTA.
-    bool ok = d.a_mn ? make_map(&g.tmA, t, d.A, d.M, d.K, d.batch, d.lda, d.strideA, 64)
-                     : make_map(&g.tmA, t, d.A, d.K, d.M, d.batch, d.lda, d.strideA, tc::BM);
-    ok = ok && (d.b_mn ? make_map(&g.tmB, t, d.B, d.N, d.K, d.batch, d.ldb, d.strideB, 64)
-                       : make_map(&g.tmB, t, d.B, d.K, d.N, d.batch, d.ldb, d.strideB, bn / pair));
-    ok = ok && make_map(&g.tmD, t, d.D, d.N, d.M, d.batch, d.ldd, d.strideD, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
-    if (!ok) return MUON_ERR_CUDA;
-    g.D = d.D;
-    g.C = d.C;
-    g.scale = d.scale;
-    g.ldd = d.ldd;
-    g.sD = d.strideD;
-    g.ldc = d.ldc;
-    g.sC = d.strideC;
-    g.M = d.M;
-    g.N = d.N;
-    g.K = d.K;
-    g.batch = d.batch;
-    g.a_mn = d.a_mn;
-    g.b_mn = d.b_mn;
-    g.sym = d.sym;
-    g.alpha_pow = d.alpha_pow;
-    g.beta_pow = d.beta_pow;
-    g.alpha = d.alpha;
-    g.beta = d.beta;
-    g.gamma = d.gamma;
-    g.tiles_m = (d.M + tile_m - 1) / tile_m;
-    g.tiles_n = (d.N + bn - 1) / bn;
-    base_tiles[i] = desc_tiles(d, tile_m, bn);
-    g.tiles_per_batch = base_tiles[i] * parts[i];
-    g.splits = parts[i];
-    g.kbps = kbps[i];
+    tc::Job& g = p.g[i];
+    if (!fill_job(g, d, t, pair, bn, parts[i], kbps[i], mt)) return MUON_ERR_CUDA;
     if (parts[i] < 2) continue;
-    const int64_t ldp = pad_ld(d.N);
-    if (!make_map(&g.tmP, Op::F32, d.part, d.N, d.M, (int64_t)parts[i] * d.batch, ldp, (int64_t)d.M * ldp, 32, 32))
-      return MUON_ERR_CUDA;
     tc::SplitGroup& r = sp.g[sp.ngroups++];
     r.part = d.part;
     r.D = d.D;
     r.C = d.C;
     r.scale = d.scale;
-    r.ldp = ldp;
+    r.ldp = pad_ld(d.N);
     r.ldd = d.ldd;
     r.sD = d.strideD;
     r.ldc = d.ldc;
@@ -1081,24 +1226,114 @@ muon_status tc_gemm(Op t, const GemmDesc* gd, int ngroups, int* status, uint64_t
   }
   p.ngroups = ng;
   p.total_tiles = total;
+  p.counters = nullptr;
   p.status = status;
-  sp.status = status;
   p.timeout_ns = timeout_ns;
+  sp.status = status;
 
   Counters& cn = counters();
   cn.launches += sp.ngroups ? 2 : 1;
   cn.gemm_launches += 1;
-  for (int i = 0; i < ng; ++i) {
-    const tc::Group& g = p.g[i];
-    const double mnk = (double)g.M * g.N * g.K * g.batch;
-    cn.flops_dense += 2.0 * mnk;
-    cn.flops_sym += g.sym ? mnk : 2.0 * mnk;
-    cn.flops_exec += 2.0 * tile_m * bn * (double)g.K * base_tiles[i] * g.batch;
-  }
+  for (int i = 0; i < ng; ++i) count_job(p.g[i], tile_m, bn);
   const muon_status r = bn == tc::BN_WIDE ? launch_for<tc::BN_WIDE>(t, pair, p, total, units, s)
                                           : launch_for<tc::BN_NARROW>(t, pair, p, total, units, s);
   if (r != MUON_OK || sp.ngroups == 0) return r;
   return t == Op::BF16 ? launch_reduce<__nv_bfloat16>(sp, red_blocks, s) : launch_reduce<__half>(sp, red_blocks, s);
+}
+
+size_t tc_chain_counter_words(int nphase, int total_batch) { return (size_t)nphase * total_batch; }
+
+muon_status tc_chain(Op t, const GemmDesc* descs, int nphase, int ngroups, unsigned* ctr, int* status,
+                     uint64_t timeout_ns, cudaStream_t s) {
+  if (nphase < 1 || ngroups < 1 || ngroups > kMaxGemmGroups || (t != Op::BF16 && t != Op::F16) || !ctr)
+    return MUON_ERR_INVALID_ARG;
+  const int pair = g_pair_mode;
+  const int tile_m = tc::BM * pair;
+  const int units_w = units_for<tc::BN_WIDE>(t, pair), units_n = units_for<tc::BN_NARROW>(t, pair);
+  if (units_w <= 0 || units_n <= 0) return MUON_ERR_CUDA;
+  int goff[kMaxGemmGroups + 1];
+  goff[0] = 0;
+  for (int i = 0; i < ngroups; ++i) {
+    for (int k = 0; k < nphase; ++k) {
+      const GemmDesc& d = descs[k * ngroups + i];
+      if (!has_work(d) || d.batch != descs[i].batch) return MUON_ERR_INVALID_ARG;
+      const muon_status c = check_desc(d);
+      if (c != MUON_OK) return c;
+    }
+    goff[i + 1] = goff[i] + descs[i].batch;
+  }
+  const int total_batch = goff[ngroups];
+
+  // One tile width for the whole chain: the one with the smaller estimated
+  // MMA time (waves of tiles times k-blocks; a 128-column k-block does half
+  // the work of a 256-column one but runs a little below half the time).
+  double cost_w = 0, cost_n = 0;
+  for (int k = 0; k < nphase; ++k) {
+    double tw = 0, tn = 0, max_kb = 0;
+    for (int i = 0; i < ngroups; ++i) {
+      const GemmDesc& d = descs[k * ngroups + i];
+      const double kb = (d.K + tc::BK - 1) / tc::BK;
+      tw += (double)desc_tiles(d, tile_m, tc::BN_WIDE) * d.batch * kb;
+      tn += (double)desc_tiles(d, tile_m, tc::BN_NARROW) * d.batch * kb;
+      max_kb = kb > max_kb ? kb : max_kb;
+    }
+    cost_w += 2.0 * std::max(tw / units_w, max_kb);
+    cost_n += 1.15 * std::max(tn / units_n, max_kb);
+  }
+  const int bn = cost_n < cost_w ? tc::BN_NARROW : tc::BN_WIDE;
+  const int units = bn == tc::BN_NARROW ? units_n : units_w;
+
+  if (cudaMemsetAsync(ctr, 0, tc_chain_counter_words(nphase, total_batch) * sizeof(unsigned), s) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  static thread_local tc::Params p;
+  static thread_local MapTable mt;
+  mt.p = &p;
+  Counters& cn = counters();
+  int k = 0;
+  while (k < nphase) {
+    // one launch: as many whole phases as its jobs and tensor maps allow
+    memset(&p, 0, sizeof(p));
+    const int k0 = k;
+    for (; k < nphase; ++k) {
+      if (p.ngroups + ngroups > tc::kMaxJobs) break;
+      const int nmaps0 = p.nmaps;
+      bool ok = true;
+      for (int i = 0; i < ngroups && ok; ++i) {
+        tc::Job& g = p.g[p.ngroups + i];
+        ok = fill_job(g, descs[k * ngroups + i], t, pair, bn, 1, (descs[k * ngroups + i].K + tc::BK - 1) / tc::BK,
+                      mt);
+        g.done = k * total_batch + goff[i];
+        if (k > k0) {
+          // the previous product of the same matrices, in this launch
+          const tc::Job& prev = p.g[p.ngroups - ngroups + i];
+          g.dep = prev.done;
+          g.dep_target = (unsigned)prev.tiles_per_batch * tc::EPI_WARPS * pair;
+        }
+      }
+      if (!ok) {
+        p.nmaps = nmaps0;  // the table is full: this phase starts the next launch
+        if (k == k0) return MUON_ERR_CUDA;
+        break;
+      }
+      p.ngroups += ngroups;
+    }
+    int total = 0;
+    for (int j = 0; j < p.ngroups; ++j) {
+      p.g[j].tile_begin = total;
+      total += p.g[j].tiles_per_batch * p.g[j].batch;
+      count_job(p.g[j], tile_m, bn);
+    }
+    p.total_tiles = total;
+    p.counters = ctr;
+    p.status = status;
+    p.timeout_ns = timeout_ns;
+    cn.launches += 1;
+    cn.gemm_launches += 1;
+    const muon_status r = bn == tc::BN_WIDE ? launch_for<tc::BN_WIDE>(t, pair, p, total, units, s)
+                                            : launch_for<tc::BN_NARROW>(t, pair, p, total, units, s);
+    if (r != MUON_OK) return r;
+  }
+  return MUON_OK;
 }
 
 }  // namespace muon

@@ -55,6 +55,23 @@ struct GemmDesc {
 // launch.
 muon_status tc_gemm(Op t, const GemmDesc* g, int ngroups, int* status, uint64_t timeout_ns, cudaStream_t s);
 
+// Fused chain: the products of a whole Newton-Schulz chain in as few
+// persistent launches as the kernel parameters allow. descs holds nphase
+// phases of ngroups products each (descs[k * ngroups + i]: phase k, shape
+// group i; every phase has the same groups and batch counts). The tiles of
+// product (k, i) for matrix b wait (bounded) until every tile of product
+// (k - 1, i) for matrix b is in memory, so the products of different matrices
+// overlap and no launch boundary separates dependent products. counters:
+// tc_chain_counter_words(nphase, sum of the groups' batch) words of
+// workspace, cleared by the call. K is never split here.
+muon_status tc_chain(Op t, const GemmDesc* descs, int nphase, int ngroups, unsigned* counters, int* status,
+                     uint64_t timeout_ns, cudaStream_t s);
+size_t tc_chain_counter_words(int nphase, int total_batch);
+
+// 1 (default 0): the Newton-Schulz chains run as fused chains (tc_chain).
+void set_gemm_chain(int on);
+int gemm_chain();
+
 // Bytes of split-K scratch that X X^T (n x n, inner dimension K) of a group
 // of `count` matrices can use in any launch; 0 when it never splits.
 size_t tc_split_scratch(int64_t n, int64_t K, int count);
@@ -100,8 +117,18 @@ struct NsGroup {
 inline int ns_work_buffers(const muon_ns_params* p) { return p->gram ? 4 : 2; }
 
 // Run the chain (standard or Gram per p->gram) on up to kMaxGemmGroups
-// groups of operand type t; all groups share each launch.
+// groups of operand type t; all groups share each launch. With the fused
+// chain on (set_gemm_chain) and `counters` non-NULL (ns_counter_words(...)
+// words of workspace), the chain's products run as one fused chain.
 muon_status ns_run(Op t, NsGroup* gs, int ng, const muon_ns_params* p, int* status, uint64_t timeout_ns,
-                   cudaStream_t s);
+                   cudaStream_t s, unsigned* counters);
+
+// Products in one chain: at most 3T (standard) or 4T + 4 (Gram with restart).
+int ns_max_phases(const muon_ns_params* p);
+// Completion-counter words a fused chain over groups holding `matrices`
+// matrices in total needs.
+inline size_t ns_counter_words(const muon_ns_params* p, int64_t matrices) {
+  return (size_t)ns_max_phases(p) * (size_t)matrices;
+}
 
 }  // namespace muon

@@ -15,6 +15,8 @@
 //   restart before step r: X <- Q X, R = rho X X^T, Q = I
 //   output Q X
 // The Frobenius scale of X_0 (xscale) enters the first products' epilogues.
+#include <vector>
+
 #include "internal.h"
 
 namespace muon {
@@ -113,7 +115,12 @@ struct Launcher {
   int* status;
   uint64_t timeout;
   cudaStream_t s;
+  std::vector<GemmDesc>* chain;  // fused chain: products are recorded, then run by tc_chain
   muon_status operator()(const GemmDesc* d, int n) const {
+    if (chain) {
+      chain->insert(chain->end(), d, d + n);
+      return MUON_OK;
+    }
     if (t == Op::F32) {
       for (int i = 0; i < n; ++i) {
         muon_status r = simt_gemm(d[i], s);
@@ -221,11 +228,23 @@ muon_status run_gram(const Launcher& L, NsGroup* gs, int ng, const muon_ns_param
 
 }  // namespace
 
+int ns_max_phases(const muon_ns_params* p) { return p->gram ? 4 * p->T + 4 : 3 * p->T; }
+
 muon_status ns_run(Op t, NsGroup* gs, int ng, const muon_ns_params* p, int* status, uint64_t timeout_ns,
-                   cudaStream_t s) {
+                   cudaStream_t s, unsigned* counters) {
   if (ng < 1 || ng > kMaxGemmGroups) return MUON_ERR_INVALID_ARG;
-  const Launcher L{t, status, timeout_ns, s};
-  return p->gram ? run_gram(L, gs, ng, p) : run_standard(L, gs, ng, p);
+  if (t == Op::F32 || !counters || !gemm_chain()) {
+    const Launcher L{t, status, timeout_ns, s, nullptr};
+    return p->gram ? run_gram(L, gs, ng, p) : run_standard(L, gs, ng, p);
+  }
+  // fused chain: record every product, then run them as one chain
+  std::vector<GemmDesc> chain;
+  const Launcher L{t, status, timeout_ns, s, &chain};
+  const muon_status r = p->gram ? run_gram(L, gs, ng, p) : run_standard(L, gs, ng, p);
+  if (r != MUON_OK || chain.empty()) return r;
+  const int nphase = (int)(chain.size() / ng);
+  if (nphase > ns_max_phases(p)) return MUON_ERR_INVALID_ARG;  // the counters are sized for ns_max_phases
+  return tc_chain(t, chain.data(), nphase, ng, counters, status, timeout_ns, s);
 }
 
 }  // namespace muon

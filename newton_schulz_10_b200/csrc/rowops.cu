@@ -272,6 +272,7 @@ __global__ void __launch_bounds__(BLOCK) update_rows(const __grid_constant__ Row
   const RowMat& m = L.m[find_mat(L, task)];
   const int64_t i = task - m.task_begin;
   if (!MUON_IN_BOUNDS(i >= 0 && i < m.ntask && m.ldx >= m.cols, L.status)) continue;
+  if (m.flag && !m.flag[i]) continue;  // a row that was not orthogonalised keeps W and M
   const int64_t j = m.idx ? (int64_t)m.idx[i] : i;
   if (!MUON_IN_BOUNDS(j >= 0 && j < m.rows, L.status)) continue;
   const float step = -L.lr * (m.rscale ? m.rscale[i] : 1.f);
@@ -302,6 +303,31 @@ __global__ void __launch_bounds__(BLOCK) update_rows(const __grid_constant__ Row
     }
   }
   report_if_any(bad, L.status);
+  }
+}
+
+// Operand rows to caller rows at their stored positions (the output of
+// muon_orthogonalize): values copied exactly (same element type).
+template <int WG, typename T>
+__global__ void __launch_bounds__(BLOCK) scatter_rows(const __grid_constant__ RowLaunch L) {
+  const int task = blockIdx.x * (BLOCK / WG) + threadIdx.x / WG;
+  const int l = threadIdx.x % WG;
+  if (task >= L.total_tasks) return;
+  const RowMat& m = L.m[find_mat(L, task)];
+  const int64_t i = task - m.task_begin;
+  if (!MUON_IN_BOUNDS(i >= 0 && i < m.ntask && m.ldx >= m.cols, L.status)) return;
+  const int64_t j = m.idx ? (int64_t)m.idx[i] : i;
+  if (!MUON_IN_BOUNDS(j >= 0 && j < m.rows, L.status)) return;
+  const T* x = reinterpret_cast<const T*>(m.X) + i * m.ldx;
+  T* o = reinterpret_cast<T*>(m.out) + j * m.cols;
+  if ((m.cols & 3) == 0) {
+    for (int64_t c = l; c < (m.cols >> 2); c += WG) Dst<T>::store4(o + 4 * c, Src<T>::load4(x + 4 * c));
+  } else {
+    for (int64_t c = l; c < m.cols; c += WG) Dst<T>::store1(o + c, Src<T>::load1(x + c));
+  }
+  if (l == 0) {
+    if (m.out_scale) m.out_scale[j] = m.rscale ? m.rscale[i] : 1.f;
+    if (m.out_flag) m.out_flag[j] = 1;
   }
 }
 
@@ -654,6 +680,19 @@ muon_status launch_update_rows(RowLaunch& L, Op ot, cudaStream_t s) {
   else if (ot == Op::F16) { if (block) UP(256, __half); else UP(32, __half); }
   else { if (block) UP(256, __nv_bfloat16); else UP(32, __nv_bfloat16); }
 #undef UP
+  return last();
+}
+
+muon_status launch_scatter_rows(RowLaunch& L, Op ot, cudaStream_t s) {
+  finish(L);
+  if (L.total_tasks == 0) return MUON_OK;
+  const bool block = use_block(L);
+  const int g = grid_for(L, block);
+#define SR(WG, T) scatter_rows<WG, T><<<g, BLOCK, 0, s>>>(L)
+  if (ot == Op::F32) { if (block) SR(256, float); else SR(32, float); }
+  else if (ot == Op::F16) { if (block) SR(256, __half); else SR(32, __half); }
+  else { if (block) SR(256, __nv_bfloat16); else SR(32, __nv_bfloat16); }
+#undef SR
   return last();
 }
 

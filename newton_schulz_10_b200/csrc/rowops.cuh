@@ -21,13 +21,19 @@ struct RowMat {
   double* rsum;           // per stored row: sum of squares (fp64)
   double* rkey;           // per stored row: selection key (fp64)
   const float* mult;      // cast multiplier (device scalar) or NULL
+  void* out;              // scatter_rows: destination rows (ld = cols), at stored row positions
+  float* out_scale;       // scatter_rows: per stored row, the update's row scale
+  int32_t* out_flag;      // scatter_rows: per stored row, 1 where the row was orthogonalised
+  const int32_t* flag;    // update: per task row, 0 = skip the row (NULL = every row)
   float kappa;            // extra cast multiplier (host constant)
   int64_t rows, cols, ldx;
   int32_t ntask;          // rows walked by this launch for this matrix
   int32_t task_begin;     // prefix of ntask over the launch's matrices
 };
 
-constexpr int kMaxRowMats = 48;
+// Matrices per row-kernel launch: the whole Llama-7B-shaped set (192) in one
+// launch; the table travels in the kernel parameters (at most 32764 bytes).
+constexpr int kMaxRowMats = 200;
 
 struct RowLaunch {
   RowMat m[kMaxRowMats];
@@ -38,6 +44,8 @@ struct RowLaunch {
   int key_l2;             // selection key: 0 = l1, 1 = sum of squares
   int* status;
 };
+
+static_assert(sizeof(RowLaunch) <= 32764, "row-kernel parameters are limited to 32764 bytes");
 
 // Kernel variants of momentum_rows.
 enum MomentumMode { MOM_MUON = 0, MOM_DION3 = 1 };
@@ -53,7 +61,11 @@ muon_status launch_cast_rows(RowLaunch& L, Op st, Op xt, cudaStream_t s);
 // rscale[i] = sum_c O[i,c]^2 (fp32), O = X of type ot.
 muon_status launch_normuon_rows(RowLaunch& L, Op ot, cudaStream_t s);
 // W[idx[i],:] -= lr * (rscale ? rscale[i] : 1) * O[i,:]; mode 1: M[idx[i],:] *= mu.
+// Rows whose flag is 0 are skipped.
 muon_status launch_update_rows(RowLaunch& L, Op ot, cudaStream_t s);
+// out[idx[i],:] = X[i,:] (type ot, ld cols), out_scale[idx[i]] = rscale ? rscale[i] : 1,
+// out_flag[idx[i]] = 1 (where non-NULL).
+muon_status launch_scatter_rows(RowLaunch& L, Op ot, cudaStream_t s);
 
 // Per-matrix scalars.
 struct NormOut {

@@ -30,7 +30,8 @@ NORM_L1, NORM_L2 = 0, 1
 EXPORTS = ("muon_set_wait_timeout_ns", "muon_set_gemm_cta_pair", "muon_status_str", "muon_rows_for_fraction", "muon_ns_params_default",
            "muon_ns_workspace_size", "ns_polar", "gram_ns_polar", "normuon_scale", "muon_select_workspace_size",
            "select_rows", "muon_workspace_size", "muon_step", "muon_step_profiled", "muon_kernel_launch_count",
-           "select_rows_noalloc", "muon_step_events")
+           "select_rows_noalloc", "muon_step_events", "muon_set_gemm_chain", "muon_momentum",
+           "muon_orthogonalize", "muon_apply_update")
 
 
 class NsParams(C.Structure):
@@ -81,6 +82,8 @@ def lib() -> C.CDLL:
         L.muon_set_wait_timeout_ns.restype = None
         L.muon_set_gemm_cta_pair.argtypes = [i32]
         L.muon_set_gemm_cta_pair.restype = None
+        L.muon_set_gemm_chain.argtypes = [i32]
+        L.muon_set_gemm_chain.restype = None
         L.muon_status_str.argtypes = [i32]
         L.muon_status_str.restype = C.c_char_p
         L.muon_rows_for_fraction.argtypes = [i64, i32, i32]
@@ -110,6 +113,14 @@ def lib() -> C.CDLL:
         L.muon_step_profiled.restype = i32
         L.muon_step_events.argtypes = [C.POINTER(Matrix), i32, C.POINTER(Params), vp, sz, vp, C.POINTER(vp)]
         L.muon_step_events.restype = i32
+        L.muon_momentum.argtypes = [C.POINTER(Matrix), i32, C.POINTER(Params), vp]
+        L.muon_momentum.restype = i32
+        L.muon_orthogonalize.argtypes = [C.POINTER(Matrix), i32, C.POINTER(Params), C.POINTER(vp), C.POINTER(vp),
+                                         C.POINTER(vp), vp, sz, vp]
+        L.muon_orthogonalize.restype = i32
+        L.muon_apply_update.argtypes = [C.POINTER(Matrix), i32, C.POINTER(Params), C.POINTER(vp), C.POINTER(vp),
+                                        C.POINTER(vp), vp]
+        L.muon_apply_update.restype = i32
         L.muon_kernel_launch_count.argtypes = []
         L.muon_kernel_launch_count.restype = i64
         _lib = L
@@ -200,6 +211,12 @@ def set_gemm_cta_pair(enable: bool) -> None:
     lib().muon_set_gemm_cta_pair(int(bool(enable)))
 
 
+def set_gemm_chain(enable: bool) -> None:
+    """True: each Newton-Schulz chain runs as one fused persistent launch;
+    False (default): one launch per product."""
+    lib().muon_set_gemm_chain(int(bool(enable)))
+
+
 def set_wait_timeout_ns(ns: int) -> None:
     lib().muon_set_wait_timeout_ns(int(ns))
 
@@ -274,7 +291,8 @@ def _matrices(mats):
     for i, m in enumerate(mats):
         W, M, G = m[0], m[1], m[2]
         v = m[3] if len(m) > 3 else None
-        arr[i] = Matrix(_ptr(W), _ptr(M), _ptr(G), _ptr(v), W.shape[0], W.shape[1])
+        shape = next(t for t in (W, M, G) if t is not None).shape
+        arr[i] = Matrix(_ptr(W), _ptr(M), _ptr(G), _ptr(v), shape[0], shape[1])
     return arr
 
 
@@ -329,6 +347,45 @@ class Step:
         if self.params.dev_status:
             raise RuntimeError("status goes to the caller's dev_status")
         return int(self.ws[:4].view(torch.int32).item())
+
+
+def _ptrs(ts):
+    arr = (C.c_void_p * max(len(ts), 1))()
+    for i, t in enumerate(ts):
+        arr[i] = _ptr(t)
+    return arr
+
+
+def operand_dtype(p: Params):
+    """torch dtype of the orthogonalised rows muon_orthogonalize writes."""
+    import torch
+    return {F32: torch.float32, BF16: torch.bfloat16, F16: torch.float16}[p.ns.compute]
+
+
+def momentum(mats, p: Params, stream=None) -> None:
+    """M <- mu M + G (M <- M + G for Dion3) on every (W, M, G[, v]) of mats."""
+    _check(lib().muon_momentum(_matrices(mats), len(mats), C.byref(p), _stream(stream)), "muon_momentum")
+
+
+def orthogonalize(mats, p: Params, O, row_scale, selected=None, ws=None, stream=None):
+    """Norms / selection, Newton-Schulz and NorMuon on the momentum of mats;
+    writes O[i] (rows x cols, operand dtype), row_scale[i] (rows) and, for
+    Dion3, selected[i] (rows, int32). Returns the workspace."""
+    table = _matrices(mats)
+    if ws is None:
+        ws = workspace(lib().muon_workspace_size(table, len(mats), C.byref(p)), mats[0][1].device if mats else None)
+    code = lib().muon_orthogonalize(table, len(mats), C.byref(p), _ptrs(O), _ptrs(row_scale),
+                                    _ptrs(selected) if selected is not None else None, _ptr(ws), ws.numel(),
+                                    _stream(stream))
+    _check(code, "muon_orthogonalize")
+    return ws
+
+
+def apply_update(mats, p: Params, O, row_scale, selected=None, stream=None) -> None:
+    """W -= lr * row_scale * O per row (Dion3: M *= mu on the selected rows)."""
+    code = lib().muon_apply_update(_matrices(mats), len(mats), C.byref(p), _ptrs(O), _ptrs(row_scale),
+                                   _ptrs(selected) if selected is not None else None, _stream(stream))
+    _check(code, "muon_apply_update")
 
 
 def muon_step(mats, p: Params | None = None, ws=None, stream=None) -> Step:
