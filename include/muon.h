@@ -239,9 +239,11 @@ muon_status select_rows(const float* M, int64_t n, int64_t m, int64_t k, muon_no
 muon_status select_rows_noalloc(const float* M, int64_t n, int64_t m, int64_t k, muon_norm norm,
                                 int32_t* idx_out, int32_t* dev_status, void* stream);
 
-/* Workspace bytes for muon_step over mats[0..count) with parameters p
- * (0 for invalid arguments). Like muon_ns_workspace_size, query with the
- * device that will run the step current. */
+/* Workspace bytes for muon_step (and muon_orthogonalize) over mats[0..count)
+ * with parameters p (0 for invalid arguments). Only the shapes and p matter:
+ * the data pointers of mats are not read and may be NULL. Like
+ * muon_ns_workspace_size, query with the device that will run the step
+ * current. */
 size_t muon_workspace_size(const muon_matrix* mats, int32_t count, const muon_params* p);
 
 /* One optimizer step over count independent matrices (host array mats):

@@ -217,8 +217,9 @@ struct StepPlan {
   size_t s, xscale, rsum, rkey, rscale, idx, ctr, total;
 };
 
-// Which fields of each muon_matrix an entry point reads.
-enum : int { NEED_W = 1, NEED_M = 2, NEED_G = 4, NEED_ALL = 7 };
+// Which fields of each muon_matrix an entry point reads (NEED_NONE: shapes
+// only, for the size queries).
+enum : int { NEED_NONE = 0, NEED_W = 1, NEED_M = 2, NEED_G = 4, NEED_V = 8, NEED_ALL = 15 };
 
 muon_status check_step(const muon_matrix* mats, int32_t count, const muon_params* p, int need = NEED_ALL) {
   if (!p || count < 0 || (count > 0 && !mats)) return MUON_ERR_INVALID_ARG;
@@ -236,7 +237,7 @@ muon_status check_step(const muon_matrix* mats, int32_t count, const muon_params
     if (m.rows < 0 || m.cols < 0 || m.rows > INT32_MAX || m.cols > INT32_MAX) return MUON_ERR_SHAPE;
     if (m.rows == 0 || m.cols == 0) continue;
     if (((need & NEED_W) && !m.W) || ((need & NEED_M) && !m.M) || ((need & NEED_G) && !m.G) ||
-        (p->normuon && !m.v))
+        ((need & NEED_V) && p->normuon && !m.v))
       return MUON_ERR_INVALID_ARG;
     if (((need & NEED_W) && !aligned16(m.W)) || ((need & NEED_M) && !aligned16(m.M)) ||
         ((need & NEED_G) && !aligned16(m.G)) || (m.v && (reinterpret_cast<uintptr_t>(m.v) & 3u)))
@@ -490,7 +491,7 @@ muon_status step_impl(const muon_matrix* mats, int32_t count, const muon_params*
 // update scales and the selection written to caller buffers.
 muon_status ortho_impl(const muon_matrix* mats, int32_t count, const muon_params* p, void* const* O,
                        float* const* row_scale, int32_t* const* selected, void* ws, size_t ws_bytes, cudaStream_t s) {
-  TRY(check_step(mats, count, p, NEED_M));
+  TRY(check_step(mats, count, p, NEED_M | NEED_V));
   if (count > 0 && (!O || !row_scale || (p->dion3 && !selected))) return MUON_ERR_INVALID_ARG;
   for (int i = 0; i < count; ++i) {
     if (mats[i].rows == 0 || mats[i].cols == 0) continue;
@@ -782,7 +783,7 @@ muon_status select_rows(const float* M, int64_t n, int64_t m, int64_t k, muon_no
 }
 
 size_t muon_workspace_size(const muon_matrix* mats, int32_t count, const muon_params* p) {
-  if (check_step(mats, count, p) != MUON_OK) return 0;
+  if (check_step(mats, count, p, NEED_NONE) != MUON_OK) return 0;
   return plan_step(mats, count, p).total;
 }
 

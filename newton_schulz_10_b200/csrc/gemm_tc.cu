@@ -49,6 +49,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cstring>
+#include <vector>
 #include <mutex>
 #include <type_traits>
 
@@ -192,6 +193,17 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t sr
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Wait until at most n (0..4) of this thread's most recent bulk groups are
+// still in flight, i.e. every older group has completed.
+__device__ __forceinline__ void bulk_wait_upto(int n) {
+  switch (n) {
+    case 4: asm volatile("cp.async.bulk.wait_group 4;" ::: "memory"); break;
+    case 3: asm volatile("cp.async.bulk.wait_group 3;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.bulk.wait_group 2;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.bulk.wait_group 1;" ::: "memory"); break;
+    default: asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); break;
+  }
+}
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // Spin (bounded) until the phase with this parity completed; for drains.
@@ -219,6 +231,13 @@ __device__ __forceinline__ void red_release_gpu_add(unsigned* a, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(a), "r"(v) : "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+__device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned* a) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+// Acquire ordering after a relaxed load that observed a released value.
+__device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 // Wait (bounded by budget) until matrix b of the job this one depends on is
 // complete. Returns false when another role raised *abort, or on expiry, in
@@ -357,6 +376,12 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     int stage = 0;
     uint32_t phase = 0;
     int issued = 0;
+    // Fused chain: the dependency counter of the next tile is read (relaxed)
+    // one tile ahead, so its latency hides behind this tile's copies; if it
+    // was already complete then, an acquire fence stands in for the acquire
+    // load, else the tile waits as usual.
+    const unsigned* next_ctr = nullptr;
+    unsigned next_val = 0;
     for (int tile = unit; tile < p.total_tiles; tile += units) {
       const Tile t = decode<PAIR, BN>(p, tile);
       const Job& g = p.g[t.g];
@@ -365,9 +390,23 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       const int am0 = t.m0 + (int)rank * BM;            // this CTA's rows of A
       const int bn0 = t.n0 + (int)rank * (BN / PAIR);   // this CTA's rows of B
       bool ok = true;
-      if (!wait_dep(p, g, t.b, abort_flag, budget)) {
-        raise_peer();
-        break;
+      if (g.dep >= 0) {
+        if (next_ctr == p.counters + g.dep + t.b && next_val >= g.dep_target) {
+          fence_acquire_gpu();
+          fence_proxy_async_global();
+        } else if (!wait_dep(p, g, t.b, abort_flag, budget)) {
+          raise_peer();
+          break;
+        }
+      }
+      next_ctr = nullptr;
+      if (tile + units < p.total_tiles) {
+        const Tile tn = decode<PAIR, BN>(p, tile + units);
+        const Job& gn = p.g[tn.g];
+        if (gn.dep >= 0) {
+          next_ctr = p.counters + gn.dep + tn.b;
+          next_val = ld_relaxed_gpu(next_ctr);
+        }
       }
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
         if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, budget, p.status)) {
@@ -505,6 +544,24 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
     uint8_t* const sm = sd + EPI_BLOCK;       // staged mirrored block
     int acc = 0;
     uint32_t acc_phase = 0;
+    // Fused chain (lane 0): the counter of this warp's last finished tile,
+    // signalled once its stores have completed. It is signalled late, after
+    // the next tile's stores are issued (their completion then overlaps that
+    // work), but always before this warp blocks on anything, so no tile
+    // waits on a signal held back by a waiting warp.
+    int pending = -1;
+    int groups = 0;  // bulk groups committed for the current tile
+    auto signal = [&]() {
+      fence_proxy_async_global();
+      red_release_gpu_add(p.counters + pending, 1u);
+      pending = -1;
+    };
+    auto flush = [&]() {
+      if (pending >= 0) {
+        bulk_wait0();
+        signal();
+      }
+    };
     for (int tile = unit; tile < p.total_tiles; tile += units) {
       const Tile t = decode<PAIR, BN>(p, tile);
       const Job& g = p.g[t.g];
@@ -525,7 +582,14 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         // C was written by an earlier product of the chain: wait for it here
         // too (these loads are issued before this tile's MMAs complete)
         bool dok = true;
-        if (lane == 0) dok = wait_dep(p, g, t.b, abort_flag, budget);
+        if (lane == 0) {
+          if (ld_acquire_gpu(p.counters + g.dep + t.b) >= g.dep_target) {
+            fence_proxy_async_global();
+          } else {
+            flush();  // this warp is about to wait: release its held signal first
+            dok = wait_dep(p, g, t.b, abort_flag, budget);
+          }
+        }
         dok = __shfl_sync(0xffffffffu, dok, 0);
         __syncwarp();  // the other lanes' loads below are ordered after lane 0's acquire
         if (!dok) {
@@ -550,6 +614,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
       }
       // every lane waits; the result is made warp-uniform so the warp-wide
       // tcgen05.ld below never runs with part of the warp gone
+      if (lane == 0 && pending >= 0 && !mbar_try_wait(smem_u32(&tfull[acc]), acc_phase)) flush();
       const bool ok = mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, budget, p.status);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) raise_peer();
@@ -579,6 +644,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
           if (lane == 0) {
             tma_store_3d(&p.maps[g.mP], smem_u32(sd), c0, r0, t.split * g.batch + t.b);
             bulk_commit();
+            ++groups;
           }
           continue;
         }
@@ -668,6 +734,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
           tma_store_3d(&p.maps[g.mD], smem_u32(sd), c0, r0, t.b);
           if (mirror) tma_store_3d(&p.maps[g.mD], smem_u32(sm), r0, c0, t.b);
           bulk_commit();
+          ++groups;
         }
       }
       // this warp's TMEM reads are done: release the accumulator (to the
@@ -678,18 +745,25 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_kernel(const __grid_constant_
         if (PAIR == 2 && rank != 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[acc]), 0));
         else mbar_arrive(&tempty[acc]);
         if (g.done >= 0) {
-          // fused chain: this warp's share of the tile is in global memory
-          bulk_wait0();
-          fence_proxy_async_global();
-          red_release_gpu_add(p.counters + g.done + t.b, 1u);
+          // fused chain: the previous tile's stores are older than this
+          // tile's `groups` bulk groups; once they completed, signal it
+          if (pending >= 0) {
+            bulk_wait_upto(groups);
+            signal();
+          }
+          pending = g.done + t.b;
         }
+        groups = 0;
       }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
       }
     }
-    if (lane == 0) bulk_wait0();  // every staged block written before the CTA exits
+    if (lane == 0) {
+      bulk_wait0();  // every staged block written before the CTA exits
+      if (pending >= 0) signal();
+    }
   }
 
   tc_fence_before();
@@ -1264,24 +1338,20 @@ muon_status tc_chain(Op t, const GemmDesc* descs, int nphase, int ngroups, unsig
   }
   const int total_batch = goff[ngroups];
 
-  // One tile width for the whole chain: the one with the smaller estimated
-  // MMA time (waves of tiles times k-blocks; a 128-column k-block does half
-  // the work of a 256-column one but runs a little below half the time).
-  double cost_w = 0, cost_n = 0;
+  // Tile width per product, by the rule of the standalone launches: 128
+  // columns when 256-column tiles leave CTAs (pairs) idle and the narrow
+  // tiles still fit in one wave. Consecutive products of one width share a
+  // launch; a change of width starts the next launch.
+  std::vector<int> bn_of(nphase);
   for (int k = 0; k < nphase; ++k) {
-    double tw = 0, tn = 0, max_kb = 0;
+    int tw = 0, tn = 0;
     for (int i = 0; i < ngroups; ++i) {
       const GemmDesc& d = descs[k * ngroups + i];
-      const double kb = (d.K + tc::BK - 1) / tc::BK;
-      tw += (double)desc_tiles(d, tile_m, tc::BN_WIDE) * d.batch * kb;
-      tn += (double)desc_tiles(d, tile_m, tc::BN_NARROW) * d.batch * kb;
-      max_kb = kb > max_kb ? kb : max_kb;
+      tw += desc_tiles(d, tile_m, tc::BN_WIDE) * d.batch;
+      tn += desc_tiles(d, tile_m, tc::BN_NARROW) * d.batch;
     }
-    cost_w += 2.0 * std::max(tw / units_w, max_kb);
-    cost_n += 1.15 * std::max(tn / units_n, max_kb);
+    bn_of[k] = (tw < units_w && tn > tw && tn <= units_n) ? tc::BN_NARROW : tc::BN_WIDE;
   }
-  const int bn = cost_n < cost_w ? tc::BN_NARROW : tc::BN_WIDE;
-  const int units = bn == tc::BN_NARROW ? units_n : units_w;
 
   if (cudaMemsetAsync(ctr, 0, tc_chain_counter_words(nphase, total_batch) * sizeof(unsigned), s) != cudaSuccess)
     return MUON_ERR_CUDA;
@@ -1291,11 +1361,14 @@ muon_status tc_chain(Op t, const GemmDesc* descs, int nphase, int ngroups, unsig
   Counters& cn = counters();
   int k = 0;
   while (k < nphase) {
-    // one launch: as many whole phases as its jobs and tensor maps allow
+    // one launch: as many whole phases of one tile width as its jobs and
+    // tensor maps allow
     memset(&p, 0, sizeof(p));
     const int k0 = k;
+    const int bn = bn_of[k0];
+    const int units = bn == tc::BN_NARROW ? units_n : units_w;
     for (; k < nphase; ++k) {
-      if (p.ngroups + ngroups > tc::kMaxJobs) break;
+      if (bn_of[k] != bn || p.ngroups + ngroups > tc::kMaxJobs) break;
       const int nmaps0 = p.nmaps;
       bool ok = true;
       for (int i = 0; i < ngroups && ok; ++i) {

@@ -99,15 +99,15 @@ def test_chain_cuda_graph_matches_eager():
     p = mu.step_params(ns=mu.ns_params(compute=mu.BF16))
     step_g = mu.Step(dm, p)
     step_e = mu.Step(de, p)
-    step_g()
+    step_g()  # first step eagerly on both (also sets kernel attributes before capture)
+    step_e()
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         step_g(torch.cuda.current_stream())
-    step_e()
-    graph.replay()
-    step_e()
-    graph.replay()
+    for _ in range(2):
+        graph.replay()
+        step_e()
     torch.cuda.synchronize()
     assert step_g.device_status() == mu.OK and step_e.device_status() == mu.OK
     for a, b in zip(dm, de):

@@ -5,6 +5,8 @@ bf16/fp16 Newton-Schulz outputs and on the weight change of a bf16 step;
 row-selection indices and the fp32 momentum state are compared bit for bit.
 """
 
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -376,10 +378,17 @@ def test_step_many_tiles_mixed_layouts(pair):
 
 
 def _launches(fn):
-    n0 = mu.kernel_launch_count()
-    out = fn()
-    torch.cuda.synchronize()
-    return out, mu.kernel_launch_count() - n0
+    """fn's result and the kernels it queued, in the per-product launch mode
+    (the split-K launches these tests count belong to that mode; the fused
+    chain never splits K)."""
+    mu.set_gemm_chain(False)
+    try:
+        n0 = mu.kernel_launch_count()
+        out = fn()
+        torch.cuda.synchronize()
+        return out, mu.kernel_launch_count() - n0
+    finally:
+        mu.set_gemm_chain(os.environ.get("MUON_GEMM_CHAIN") == "1")
 
 
 @pytest.mark.parametrize("pair", [True, False])
