@@ -253,9 +253,19 @@ def measured_peaks():
 
 
 def use_graph(args, big: bool) -> bool:
-    """CUDA-graph replay for the small layer sets (launch-bound), eager
-    launches with per-step phase events for the large ones."""
+    """The small layer sets (a few ms per step, tens of launches) replay the
+    step as a captured CUDA graph, which takes the host out of the loop; the
+    large ones run eager steps that record their own phase events, queued
+    behind a short device-side sleep so the GPU runs them back to back."""
     return bool(args.graph) if args.graph >= 0 else not big
+
+
+PRIME_CYCLES = 4_000_000  # ~2-3 ms of device time: the host queues the timed steps meanwhile
+
+
+def prime(torch):
+    """Keep the stream busy while the host queues the timed region."""
+    torch.cuda._sleep(PRIME_CYCLES)
 
 
 def config_for(args, specs=None) -> dict:
@@ -271,7 +281,7 @@ def config_for(args, specs=None) -> dict:
     big = elems > 1_000_000_000
     return {"workload": args.workload, "description": cfg["desc"], "matrices": len(specs), "elements": elems,
             "state_bytes": 12 * elems, "l2": "inputs larger than L2 (fp32 W, M, G resident in HBM)",
-            "execution": "cuda_graph" if use_graph(args, big) else "eager, phase events per step",
+            "execution": "cuda_graph" if use_graph(args, big) else "eager, queued behind a device sleep, phase events per step",
             "parallelism": "replicas" if args.gpus > 1 else "single GPU"}
 
 
@@ -452,6 +462,7 @@ def run_ours(args, rank, world, local_rank):
                 graph.replay()
             e1.record(stream)
         else:
+            prime(torch)
             evs, e0, e1 = timed_eager(step, stream, args.steps, torch)
         torch.cuda.synchronize()
         t1 = time.time()
@@ -464,15 +475,20 @@ def run_ours(args, rank, world, local_rank):
     clocks = clk.summary(t0, t1)
     status = step.device_status()
 
-    # --- phases: from the timed steps' own events (eager), else from a
-    # profiled eager step of the same run (graph replays cannot be bracketed)
-    if evs is not None:
-        ph = phase_means(evs)
-        ph = {k: max_over_ranks(v, world) for k, v in ph.items()}
-        phase_src = "CUDA events of the timed steps (muon_step_events), mean over steps, max over ranks"
+    # --- phases: from the timed steps' own events (eager); after graph
+    # replays (which cannot be bracketed) from as many eager steps of the same
+    # workload, queued behind a device sleep, right after the timed region
+    if evs is None:
+        if world > 1:
+            dist.barrier()
+        prime(torch)
+        evs, _, _ = timed_eager(step, stream, args.steps, torch)
+        torch.cuda.synchronize()
+        phase_src = (f"CUDA events of {args.steps} eager steps (muon_step_events, queued behind a device sleep) "
+                     "run after the timed graph replays, mean over steps, max over ranks")
     else:
-        ph = {k: getattr(prof, k) for k in ("ms_total", "ms_prologue", "ms_ns", "ms_normuon", "ms_update")}
-        phase_src = "CUDA events of a profiled eager step in the same run (the timed region replays a graph)"
+        phase_src = "CUDA events of the timed steps (muon_step_events), mean over steps, max over ranks"
+    ph = {k: max_over_ranks(v, world) for k, v in phase_means(evs).items()}
 
     peaks, peak_kind = measured_peaks()
     long_step = ms > 100.0
@@ -511,6 +527,7 @@ def run_ours(args, rank, world, local_rank):
         profn = stepn.profiled(stream)
         if world > 1:
             dist.barrier()
+        prime(torch)
         evn, n0e, n1e = timed_eager(stepn, stream, kn, torch)
         torch.cuda.synchronize()
         msn = max_over_ranks(n0e.elapsed_time(n1e) / kn, world)
@@ -593,6 +610,7 @@ def run_spectrum(args, rank, world, local_rank):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with ClockSampler(local_rank) as clk:
             t0 = time.time()
+            prime(torch)
             e0.record(stream)
             for _ in range(args.steps):
                 O, _ = mu.ns_polar(Xd, p, out_dtype=torch.bfloat16, ws=ws)
@@ -739,11 +757,11 @@ def threads_used():
 
 
 def run_reference(args):
-    """The reference arm: the fp64 CPU oracle as it stands. Each step (warm-up
-    or timed) times one matrix, the distinct shapes taken in turn, and reports
-    the whole-step estimate from every shape's mean time so far; the warm-up
-    steps (at least one per shape) give every shape a time before the first
-    timed step."""
+    """The reference arm: the fp64 CPU oracle as it stands. Each timed step
+    times one matrix, the distinct shapes taken in turn, and reports the
+    whole-step estimate from every shape's mean time so far; the warm-up
+    times one matrix of every shape, so that every shape has a time before
+    the first timed step."""
     vals = []
     if args.workload in SPECTRUM:
         for _ in range(args.warmup):
@@ -754,7 +772,9 @@ def run_reference(args):
     else:
         smp = OracleSampler(args.workload)
         k = 0
-        for _ in range(max(args.warmup, len(smp.shapes))):
+        # warm-up: one sample per distinct shape (numpy has nothing to warm;
+        # these give every shape a time before the first timed step)
+        for _ in range(len(smp.shapes)):
             smp.time_shape(k)
             k += 1
         for _ in range(args.steps):
@@ -789,7 +809,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end arm")
     ap.add_argument("--no-normuon", action="store_true", help="skip the NorMuon-on timing of the Llama-7B set")
     ap.add_argument("--graph", type=int, default=-1,
-                    help="1: replay the step as one captured CUDA graph, 0: eager with per-step phase events, "
+                    help="1: replay the step as one captured CUDA graph (phases then from as many eager steps), "
+                         "0: eager steps queued behind a device-side sleep, each recording its own phase events, "
                          "-1 (default): graph for the small layer sets, eager for the large ones")
     ap.add_argument("--cta-pair", type=int, default=1, help="1: CTA-pair tensor-core GEMM, 0: single-CTA")
     ap.add_argument("--wait-timeout-ms", type=float, default=0.0, help="bound of device-side waits (0: default)")

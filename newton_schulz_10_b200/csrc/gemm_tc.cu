@@ -1342,6 +1342,9 @@ muon_status tc_chain(Op t, const GemmDesc* descs, int nphase, int ngroups, unsig
   // columns when 256-column tiles leave CTAs (pairs) idle and the narrow
   // tiles still fit in one wave. Consecutive products of one width share a
   // launch; a change of width starts the next launch.
+  // A product that the standalone launch would split along K (an X X^T
+  // with a long K and fewer tiles than CTA pairs) runs as that split launch
+  // (bn_of = 0): the chain stops before it and resumes after it.
   std::vector<int> bn_of(nphase);
   for (int k = 0; k < nphase; ++k) {
     int tw = 0, tn = 0;
@@ -1350,7 +1353,14 @@ muon_status tc_chain(Op t, const GemmDesc* descs, int nphase, int ngroups, unsig
       tw += desc_tiles(d, tile_m, tc::BN_WIDE) * d.batch;
       tn += desc_tiles(d, tile_m, tc::BN_NARROW) * d.batch;
     }
-    bn_of[k] = (tw < units_w && tn > tw && tn <= units_n) ? tc::BN_NARROW : tc::BN_WIDE;
+    bool split = false;
+    for (int i = 0; i < ngroups; ++i) {
+      const GemmDesc& d = descs[k * ngroups + i];
+      int per = 0;
+      const int parts = d.sym && d.part ? split_parts(tw, units_w, (d.K + tc::BK - 1) / tc::BK, &per) : 1;
+      split = split || (parts > 1 && (size_t)parts * d.batch * d.N * pad_ld(d.N) * sizeof(float) <= d.part_bytes);
+    }
+    bn_of[k] = split ? 0 : (tw < units_w && tn > tw && tn <= units_n) ? tc::BN_NARROW : tc::BN_WIDE;
   }
 
   if (cudaMemsetAsync(ctr, 0, tc_chain_counter_words(nphase, total_batch) * sizeof(unsigned), s) != cudaSuccess)
@@ -1361,6 +1371,12 @@ muon_status tc_chain(Op t, const GemmDesc* descs, int nphase, int ngroups, unsig
   Counters& cn = counters();
   int k = 0;
   while (k < nphase) {
+    if (bn_of[k] == 0) {
+      const muon_status r = tc_gemm(t, descs + k * ngroups, ngroups, status, timeout_ns, s);
+      if (r != MUON_OK) return r;
+      ++k;
+      continue;
+    }
     // one launch: as many whole phases of one tile width as its jobs and
     // tensor maps allow
     memset(&p, 0, sizeof(p));

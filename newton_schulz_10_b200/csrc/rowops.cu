@@ -4,6 +4,8 @@
 // finalisers. Rows are walked by a warp (short rows) or a whole block (long
 // rows) with 16-byte vector accesses when the row length allows; every
 // reduction runs in a fixed order, so results are bit-reproducible.
+#include <mutex>
+
 #include "common.cuh"
 #include "rowops.cuh"
 
@@ -354,19 +356,29 @@ __global__ void __launch_bounds__(BLOCK) norm_finalize(const __grid_constant__ F
 }
 
 constexpr int SEL_THREADS = 1024;
+// Keys of up to this many rows are staged in shared memory once (8 bytes
+// each) and every radix pass reads them there; longer key arrays are read
+// from global memory in every pass.
+constexpr int64_t SEL_SMEM_ROWS = 20480;
 
 // Top-k by radix selection on the fp64 key bits (keys are >= 0, so their bit
 // patterns order like the values), then an index-ordered compaction.
 __global__ void __launch_bounds__(SEL_THREADS) select_topk(const double* key, const double* rsum, int64_t n,
                                                            int64_t k, int32_t* idx, float* s_out, float* xscale_out,
                                                            float eps, float inv_kappa, int* status) {
+  extern __shared__ unsigned long long skeys[];
   __shared__ unsigned int hist[256];
   __shared__ unsigned long long s_prefix;
   __shared__ long long s_remaining;
   __shared__ long long warp_cnt[SEL_THREADS / 32];
   __shared__ double scratch[32];
   const int tid = threadIdx.x;
+  const bool staged = n <= SEL_SMEM_ROWS;
   const unsigned long long* u = reinterpret_cast<const unsigned long long*>(key);
+  if (staged) {
+    for (int64_t i = tid; i < n; i += SEL_THREADS) skeys[i] = u[i];
+    u = skeys;
+  }
   if (tid == 0) {
     s_prefix = 0ull;
     s_remaining = k;
@@ -381,18 +393,39 @@ __global__ void __launch_bounds__(SEL_THREADS) select_topk(const double* key, co
       if ((x & mask) == prefix) atomicAdd(&hist[(x >> shift) & 255ull], 1u);
     }
     __syncthreads();
-    if (tid == 0) {
-      long long rem = s_remaining, cum = 0;
-      int sel = 0;
-      for (int d = 255; d >= 0; --d) {
-        if (cum + (long long)hist[d] >= rem) {
-          sel = d;
-          break;
-        }
-        cum += hist[d];
+    if (tid < 32) {
+      // the digit of the k-th largest key among those with this prefix: lane
+      // l holds bins 255 - 8l down to 248 - 8l, an inclusive scan over lanes
+      // counts the keys at or above each lane's bins, and the first lane
+      // whose count reaches the remaining rank finds the digit in its bins
+      unsigned c[8], tot = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c[j] = hist[255 - 8 * tid - j];
+        tot += c[j];
       }
-      s_remaining = rem - cum;
-      s_prefix = prefix | ((unsigned long long)sel << shift);
+      unsigned incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += y;
+      }
+      const long long rem = s_remaining;
+      const unsigned hit = __ballot_sync(0xffffffffu, (long long)incl >= rem);
+      if (tid == __ffs(hit) - 1) {
+        long long cum = (long long)(incl - tot);  // keys above this lane's bins
+        int sel = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (cum + (long long)c[j] >= rem) {
+            sel = 255 - 8 * tid - j;
+            break;
+          }
+          cum += c[j];
+        }
+        s_remaining = rem - cum;
+        s_prefix = prefix | ((unsigned long long)sel << shift);
+      }
     }
     mask |= 255ull << shift;
     __syncthreads();
@@ -708,7 +741,26 @@ muon_status launch_norm_finalize(const NormOut* out, int count, float eps, int* 
 
 muon_status launch_select(const double* key, const double* rsum, int64_t n, int64_t k, int32_t* idx, float* s_out,
                           float* xscale_out, float eps, float inv_kappa, int* status, cudaStream_t s) {
-  select_topk<<<1, SEL_THREADS, 0, s>>>(key, rsum, n, k, idx, s_out, xscale_out, eps, inv_kappa, status);
+  // the staged keys need more than the default 48 KB of dynamic shared
+  // memory: allowed once per device
+  static std::mutex mu;
+  static bool set_up[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return MUON_ERR_CUDA;
+  }
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!set_up[dev]) {
+      if (cudaFuncSetAttribute((const void*)select_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)(SEL_SMEM_ROWS * sizeof(unsigned long long))) != cudaSuccess)
+        return MUON_ERR_CUDA;
+      set_up[dev] = true;
+    }
+  }
+  const size_t smem = n <= SEL_SMEM_ROWS ? (size_t)n * sizeof(unsigned long long) : 0;
+  select_topk<<<1, SEL_THREADS, smem, s>>>(key, rsum, n, k, idx, s_out, xscale_out, eps, inv_kappa, status);
   return last();
 }
 

@@ -336,6 +336,11 @@ class Step:
         `events` (enable_timing=True) at its phase boundaries on the stream:
         start, NS chain start, NS chain end, NorMuon end, update end. Does not
         synchronise."""
+        import torch
+        ts = stream if stream is not None else torch.cuda.current_stream()
+        for e in events:
+            if not e.cuda_event:  # torch creates the CUDA event at its first record
+                e.record(ts)
         handles = (C.c_void_p * 5)(*[e.cuda_event for e in events])
         code = lib().muon_step_events(self._table, len(self.mats), C.byref(self.params), _ptr(self.ws),
                                       self.ws.numel(), _stream(stream), handles)

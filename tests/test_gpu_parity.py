@@ -519,3 +519,27 @@ def test_nonfinite_output_is_reported(gram):
     state = make_state([(256, 1024)], 9710, m_std=1e-3)
     _, st = run_step(state, mu.step_params(ns=mu.ns_params(T=3, coeffs=table, gram=gram, compute=mu.F16)))
     assert st == mu.ERR_NONFINITE
+
+
+def test_step_events_record_phases():
+    """muon_step_events records the caller's five events at the phase
+    boundaries of an ordinary step (fresh torch events included: they get a
+    CUDA handle before the call), without changing the step: the state equals
+    a muon_step run's bit for bit, and the phase times are positive and add up
+    to the span of the first and last event."""
+    state = make_state(MIXED, 7800, m_std=1e-3)
+    p = mu.step_params(normuon=True)
+    d1 = [(dev(W), dev(M), dev(G), dev(v)) for (W, M, G, v) in state]
+    d2 = [tuple(t.clone() for t in m) for m in d1]
+    mu.muon_step(d1, p)
+    s2 = mu.Step(d2, p)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    s2.timed(ev)
+    torch.cuda.synchronize()
+    assert s2.device_status() == mu.OK
+    for a, b in zip(d1, d2):
+        for x, y in zip(a, b):
+            assert torch.equal(x, y)
+    phases = [ev[i].elapsed_time(ev[i + 1]) for i in range(4)]
+    assert phases[1] > 0 and all(t >= 0 for t in phases)
+    assert abs(sum(phases) - ev[0].elapsed_time(ev[4])) < 1e-3 * max(1.0, sum(phases))
