@@ -10,9 +10,9 @@ times (all matrices of a layer set in one batched step).
   result; bounded by the oracle's own half-precision emulation at this size
   (tests/golden/spectrum_4096x16384_emulated.json) and exact to 2e-2 on the
   well-conditioned directions.
-- Llama-7B layer set: the whole 192-matrix step on the GPU, layer 0 (six
-  matrices, drawn by the NumPy recipe) checked against the oracle; the other
-  layers are drawn on the device.
+- Llama-7B layer set, NorMuon off and on: the whole 192-matrix step on the
+  GPU, layer 0 (six matrices, drawn by the NumPy recipe) checked against the
+  oracle; the other layers are drawn on the device.
 """
 
 import json
@@ -132,7 +132,11 @@ def _spectrum_exact(X32):
     return _EXACT[key]
 
 
-def test_llama7b_sampled_layer0():
+@pytest.mark.parametrize("normuon", [False, True], ids=["normuon_off", "normuon_on"])
+def test_llama7b_sampled_layer0(normuon):
+    """The Llama-7B workload with NorMuon off and then on (Eq. (2) on every
+    row, v from zero): the whole 192-matrix step on the GPU, layer 0 against
+    the oracle (momentum bit for bit, dW and v within 2e-2)."""
     specs = inputs.llama7b_layer_set()
     layer0 = [s for s in specs if s.name.startswith("l0.")]
     host_state = {}
@@ -150,11 +154,11 @@ def test_llama7b_sampled_layer0():
             W = torch.randn(shape, device="cuda", generator=g) * 0.02
             G = torch.randn(shape, device="cuda", generator=g) * 1e-3
             dmats.append((W, torch.zeros(shape, device="cuda"), G, torch.zeros(s.rows, device="cuda")))
-    step = mu.muon_step(dmats, mu.step_params())
+    step = mu.muon_step(dmats, mu.step_params(normuon=normuon, beta2=0.95, normuon_eps=1e-8))
     assert step.device_status() == mu.OK
     got = {s.name: (d[0].cpu().numpy(), d[1].cpu().numpy(), d[3].cpu().numpy())
            for s, d in zip(specs, dmats) if s.name.startswith("l0.")}
     del dmats, step
     for s in layer0:
-        e = _check_matrix(*host_state[s.name], got[s.name], O.StepParams(), s.name)
-        print(f"llama7b {s.name}: relative dW error {e:.3e}")
+        e = _check_matrix(*host_state[s.name], got[s.name], O.StepParams(normuon=normuon), s.name)
+        print(f"llama7b {s.name} (NorMuon {'on' if normuon else 'off'}): relative dW error {e:.3e}")
