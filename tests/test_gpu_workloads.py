@@ -50,7 +50,11 @@ def _check_matrix(W, M, G, v, got, sp, label):
     e = rel(dW, dW_want)
     assert e < TOL16, (label, e)
     if sp.normuon:
-        assert rel(vg, want["v"]) < TOL16, label
+        # v_i = beta2 v_i + (1 - beta2) sum_j O_ij^2 / m is quadratic in the
+        # Newton-Schulz output: a relative error eps in O's rows is about
+        # 2 eps in v, so the 2e-2 bound of half-precision NS outputs is 4e-2
+        # here
+        assert rel(vg, want["v"]) < 2 * TOL16, (label, rel(vg, want["v"]))
     return e
 
 
