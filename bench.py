@@ -308,10 +308,13 @@ def end_to_end(args, state, step, stream, elems, big, world):
     except ImportError:
         avail = 1 << 62
     free_dev, _ = torch.cuda.mem_get_info()
-    if 8 * elems > 0.5 * avail or 8 * elems > 0.9 * free_dev:
+    # every rank on this node pins its own G and W copies at the same time
+    ranks_here = int(os.environ.get("LOCAL_WORLD_SIZE", "1"))
+    if 8 * elems * ranks_here > 0.5 * avail or 8 * elems > 0.9 * free_dev:
         return {"value": None, "unit": "ms/step", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "reason": f"needs {8 * elems / 1e9:.1f} GB pinned host and device memory "
-                          f"({avail / 1e9:.1f} GB host available, {free_dev / 1e9:.1f} GB device free)"}
+                "reason": f"needs {8 * elems / 1e9:.1f} GB pinned host memory per rank ({ranks_here} ranks on "
+                          f"this node) and as much device memory ({avail / 1e9:.1f} GB host available, "
+                          f"{free_dev / 1e9:.1f} GB device free)"}
     hostG = [torch.empty_like(G, device="cpu").pin_memory() for (_, _, G, _) in state]
     for hg, (_, _, G, _) in zip(hostG, state):
         hg.copy_(G)
