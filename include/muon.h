@@ -264,7 +264,8 @@ muon_status muon_step(const muon_matrix* mats, int32_t count, const muon_params*
  * muon_momentum: the first line of Eq. (1) on every matrix, elementwise:
  * M <- mu M + G (one rounding, as a fused multiply-add), or M <- M + G when
  * p->dion3 (Algorithm 4 keeps the decay for the error feedback). Reads M and
- * G, writes M; W and v are not touched. No workspace. */
+ * G, writes M; W and v are not touched. No workspace, no deferred errors
+ * (a non-finite M surfaces in muon_orthogonalize). */
 muon_status muon_momentum(const muon_matrix* mats, int32_t count, const muon_params* p, void* stream);
 
 /* muon_orthogonalize: everything between the momentum and the weight update,
@@ -281,7 +282,9 @@ muon_status muon_momentum(const muon_matrix* mats, int32_t count, const muon_par
  *   selected[i]   rows int32 (needed when p->dion3, else may be NULL): 1 for
  *                 the selected rows, 0 elsewhere
  * so that the update is W[r,:] -= lr * row_scale[i][r] * O[i][r,:].
- * ws / ws_bytes: as for muon_step (muon_workspace_size). */
+ * ws / ws_bytes: as for muon_step (muon_workspace_size). Deferred errors (a
+ * non-finite norm or NorMuon ratio, a bounded wait that ran out) go to
+ * p->dev_status, else to the first 4 workspace bytes, as for muon_step. */
 muon_status muon_orthogonalize(const muon_matrix* mats, int32_t count, const muon_params* p,
                                void* const* O, float* const* row_scale, int32_t* const* selected,
                                void* ws, size_t ws_bytes, void* stream);
@@ -291,7 +294,9 @@ muon_status muon_orthogonalize(const muon_matrix* mats, int32_t count, const muo
  * whose O, row_scale and selected rows are passed for the same range):
  * W[r,:] <- W[r,:] - lr * row_scale[i][r] * O[i][r,:] (one rounding), and,
  * when p->dion3, M[r,:] <- mu M[r,:] for the selected rows, whose W alone
- * changes. Reads O, row_scale, selected; G and v are not touched. */
+ * changes. Reads O, row_scale, selected; G and v are not touched. A
+ * non-finite value of O is reported as MUON_ERR_NONFINITE to p->dev_status
+ * when it is set (no workspace, so nothing is reported without it). */
 muon_status muon_apply_update(const muon_matrix* mats, int32_t count, const muon_params* p,
                               const void* const* O, const float* const* row_scale,
                               const int32_t* const* selected, void* stream);
