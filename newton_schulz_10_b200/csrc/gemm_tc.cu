@@ -101,6 +101,7 @@ struct Job {
   long long ldd, sD, ldc, sC;
   int M, N, K, batch;
   int a_mn, b_mn, sym;
+  int n_fast;  // non-symmetric tile order: 1 = N fastest, 0 = M fastest
   int alpha_pow, beta_pow;
   float alpha, beta, gamma;
   int tiles_m, tiles_n, tiles_per_batch, tile_begin;  // tiles_per_batch counts (tile, split) units
@@ -154,8 +155,18 @@ __device__ inline Tile decode(const Params& p, int tile) {
   t /= g.splits;
   int tm, tn;
   if (!g.sym) {
-    tm = t % g.tiles_m;  // M fastest: concurrent CTAs share the B column block
-    tn = t / g.tiles_m;
+    // The fastest dimension cycles through the smaller operand's panels,
+    // which stay in L2, while the slow one walks the larger operand's panels
+    // so that each is read from memory once; the other order would re-read
+    // the whole larger operand every wave (for a tall X times a square P,
+    // far more than L2 holds).
+    if (g.n_fast) {
+      tn = t % g.tiles_n;
+      tm = t / g.tiles_n;
+    } else {
+      tm = t % g.tiles_m;
+      tn = t / g.tiles_m;
+    }
   } else {
     int i = 0;
     for (;;) {
@@ -1168,6 +1179,7 @@ bool fill_job(tc::Job& g, const GemmDesc& d, Op t, int pair, int bn, int parts, 
   g.a_mn = d.a_mn;
   g.b_mn = d.b_mn;
   g.sym = d.sym;
+  g.n_fast = !d.sym && d.N < d.M ? 1 : 0;  // B (N x K) is the smaller operand
   g.alpha_pow = d.alpha_pow;
   g.beta_pow = d.beta_pow;
   g.alpha = d.alpha;
