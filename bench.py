@@ -54,6 +54,9 @@ WORKLOADS = {
                                  compute="bf16", gram=False, normuon=False, dion3=None),
     "llama7b_normuon": dict(desc="Llama-7B layer set, bf16 NS T=5, NorMuon on",
                             compute="bf16", gram=False, normuon=True, dion3=None),
+    "llama7b_gram": dict(desc="Llama-7B layer set, Gram NS fp16 (restart 3), T=5: the Gram reformulation on "
+                              "the same 192 matrices",
+                         compute="f16", gram=True, normuon=False, dion3=None),
     "spectrum4096x16384": dict(desc="one 4096x16384 bf16 matrix, singular values log-uniform in [1e-4, 1]: "
                                     "Gram NS (fp16, restart 3) vs standard NS (bf16 and fp16), T=5",
                                compute="f16", gram=True, normuon=False, dion3=None),

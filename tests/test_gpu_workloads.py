@@ -136,11 +136,13 @@ def _spectrum_exact(X32):
     return _EXACT[key]
 
 
-@pytest.mark.parametrize("normuon", [False, True], ids=["normuon_off", "normuon_on"])
-def test_llama7b_sampled_layer0(normuon):
+@pytest.mark.parametrize("normuon,gram", [(False, False), (True, False), (False, True)],
+                         ids=["normuon_off", "normuon_on", "gram_f16"])
+def test_llama7b_sampled_layer0(normuon, gram):
     """The Llama-7B workload with NorMuon off and then on (Eq. (2) on every
-    row, v from zero): the whole 192-matrix step on the GPU, layer 0 against
-    the oracle (momentum bit for bit, dW and v within 2e-2)."""
+    row, v from zero), and with Gram Newton-Schulz in fp16 (restart 3): the
+    whole 192-matrix step on the GPU, layer 0 against the oracle (momentum
+    bit for bit, dW and v within 2e-2)."""
     specs = inputs.llama7b_layer_set()
     layer0 = [s for s in specs if s.name.startswith("l0.")]
     host_state = {}
@@ -158,11 +160,13 @@ def test_llama7b_sampled_layer0(normuon):
             W = torch.randn(shape, device="cuda", generator=g) * 0.02
             G = torch.randn(shape, device="cuda", generator=g) * 1e-3
             dmats.append((W, torch.zeros(shape, device="cuda"), G, torch.zeros(s.rows, device="cuda")))
-    step = mu.muon_step(dmats, mu.step_params(normuon=normuon, beta2=0.95, normuon_eps=1e-8))
+    ns = mu.ns_params(gram=True, restart_at=3, compute=mu.F16) if gram else mu.ns_params()
+    step = mu.muon_step(dmats, mu.step_params(ns=ns, normuon=normuon, beta2=0.95, normuon_eps=1e-8))
     assert step.device_status() == mu.OK
     got = {s.name: (d[0].cpu().numpy(), d[1].cpu().numpy(), d[3].cpu().numpy())
            for s, d in zip(specs, dmats) if s.name.startswith("l0.")}
     del dmats, step
     for s in layer0:
-        e = _check_matrix(*host_state[s.name], got[s.name], O.StepParams(normuon=normuon), s.name)
-        print(f"llama7b {s.name} (NorMuon {'on' if normuon else 'off'}): relative dW error {e:.3e}")
+        e = _check_matrix(*host_state[s.name], got[s.name], O.StepParams(normuon=normuon, gram=gram), s.name)
+        label = "Gram fp16" if gram else f"NorMuon {'on' if normuon else 'off'}"
+        print(f"llama7b {s.name} ({label}): relative dW error {e:.3e}")
