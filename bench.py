@@ -566,7 +566,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches,
         "clocks": clocks,
         "device_status": mu.status_str(status),
-        "gemm": "cta_pair" if args.cta_pair else "single_cta",
+        "gemm": ("cta_pair" if args.cta_pair else "single_cta") + (", fused chain" if args.gemm_chain else ""),
     }
     return out
 
@@ -822,6 +822,9 @@ def main():
                          "0: eager steps queued behind a device-side sleep, each recording its own phase events, "
                          "-1 (default): graph for the small layer sets, eager for the large ones")
     ap.add_argument("--cta-pair", type=int, default=1, help="1: CTA-pair tensor-core GEMM, 0: single-CTA")
+    ap.add_argument("--gemm-chain", type=int, default=0,
+                    help="1: run each Newton-Schulz chain as one fused persistent launch (completion counters "
+                         "between dependent products), 0: one launch per product")
     ap.add_argument("--wait-timeout-ms", type=float, default=0.0, help="bound of device-side waits (0: default)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -844,6 +847,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     from newton_schulz_10_b200 import muon as mu
     mu.set_gemm_cta_pair(bool(args.cta_pair))
+    mu.set_gemm_chain(bool(args.gemm_chain))
     if args.wait_timeout_ms > 0:
         mu.set_wait_timeout_ns(int(args.wait_timeout_ms * 1e6))
     if args.workload in SPECTRUM:
