@@ -57,6 +57,9 @@ WORKLOADS = {
     "llama7b_gram": dict(desc="Llama-7B layer set, Gram NS fp16 (restart 3), T=5: the Gram reformulation on "
                               "the same 192 matrices",
                          compute="f16", gram=True, normuon=False, dion3=None),
+    "llama7b_gram_layer": dict(desc="one layer of the Llama-7B set, Gram NS fp16 (restart 3), T=5 (profiling case: "
+                                    "per-launch traffic x 32 = the full set's)",
+                               compute="f16", gram=True, normuon=False, dion3=None),
     "spectrum4096x16384": dict(desc="one 4096x16384 bf16 matrix, singular values log-uniform in [1e-4, 1]: "
                                     "Gram NS (fp16, restart 3) vs standard NS (bf16 and fp16), T=5",
                                compute="f16", gram=True, normuon=False, dion3=None),
@@ -90,7 +93,7 @@ def specs_for(name: str):
         return [inputs.MatrixSpec(8192, 28672, 4000, "x")]
     if name == "llama_mlp_4096x14336":
         return [inputs.llama7b_layer_set()[4]]
-    if name == "llama7b_layer":
+    if name in ("llama7b_layer", "llama7b_gram_layer"):
         return inputs.llama7b_layer_set(layers=1)
     if name.startswith("llama7b"):
         return inputs.llama7b_layer_set()
